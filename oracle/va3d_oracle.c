@@ -152,18 +152,27 @@ int oracle_rope3d(const uint16_t *x, double *y, long BH, long N, int head_dim,
     return ORACLE_OK;
 }
 
-/* Whether query token i may attend to key token j in the given mode.
- *  full:     every token attends to every token (joint video+text too);
- *  spatial:  tokens of the same frame t;
- *  temporal: tokens of the same spatial position (h, w). */
-static int allowed(const oracle_grid *g, int mode, long i, long j)
+/* The keys query token i attends to, following the handbook's section "How
+ * attention sees time": full attention takes every token (joint video+text
+ * too); the spatial pass takes the H'W' tokens of i's frame; the temporal pass
+ * takes the T' tokens at i's spatial position (h, w), one per frame.
+ * Writes the key indices to keys[] and returns their count. */
+static long key_set(const oracle_grid *g, int mode, long i, long N, long *keys)
 {
-    if (mode == ORACLE_FULL) return 1;
-    int ti, hi, wi, tj, hj, wj;
-    oracle_token_coords(g, i, &ti, &hi, &wi);
-    oracle_token_coords(g, j, &tj, &hj, &wj);
-    if (mode == ORACLE_SPATIAL) return ti == tj;
-    return hi == hj && wi == wj;
+    long cnt = 0;
+    if (mode == ORACLE_FULL) {
+        for (long j = 0; j < N; ++j) keys[cnt++] = j;
+        return cnt;
+    }
+    int t, h, w;
+    oracle_token_coords(g, i, &t, &h, &w);
+    const long hw = (long)g->H * g->W;
+    if (mode == ORACLE_SPATIAL) {
+        for (long j = 0; j < hw; ++j) keys[cnt++] = (long)t * hw + j;
+    } else {
+        for (long tt = 0; tt < g->T; ++tt) keys[cnt++] = tt * hw + (long)h * g->W + w;
+    }
+    return cnt;
 }
 
 /*
@@ -226,6 +235,7 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             double *qr = (double *)malloc(sizeof(double) * D);
             double *qx = (double *)malloc(sizeof(double) * D);
             double *s = (double *)malloc(sizeof(double) * (size_t)N);
+            long *keys = (long *)malloc(sizeof(long) * (size_t)N);
             double *acc = (double *)malloc(sizeof(double) * D);
 #pragma omp for schedule(dynamic, 1)
             for (long r = 0; r < nrows; ++r) {
@@ -235,24 +245,25 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                     rope_row(g, head_dim, qx, qr, i);
                 else
                     memcpy(qr, qx, sizeof(double) * D);
+                const long nk = key_set(g, mode, i, N, keys);
 
-                /* scores and their maximum over the allowed keys */
+                /* scores and their maximum over the keys */
                 double m = -INFINITY;
-                for (long j = 0; j < N; ++j) {
-                    if (!allowed(g, mode, i, j)) continue;
+                for (long e = 0; e < nk; ++e) {
+                    const double *kj = kr + keys[e] * D;
                     double dot = 0.0;
-                    for (size_t c = 0; c < D; ++c) dot += qr[c] * kr[j * D + c];
-                    s[j] = dot * scale;
-                    if (s[j] > m) m = s[j];
+                    for (size_t c = 0; c < D; ++c) dot += qr[c] * kj[c];
+                    s[e] = dot * scale;
+                    if (s[e] > m) m = s[e];
                 }
                 /* normalised weighted sum of values */
                 double z = 0.0;
                 for (size_t c = 0; c < D; ++c) acc[c] = 0.0;
-                for (long j = 0; j < N; ++j) {
-                    if (!allowed(g, mode, i, j)) continue;
-                    double p = exp(s[j] - m);
+                for (long e = 0; e < nk; ++e) {
+                    double p = exp(s[e] - m);
+                    const double *vj = vd + keys[e] * D;
                     z += p;
-                    for (size_t c = 0; c < D; ++c) acc[c] += p * vd[j * D + c];
+                    for (size_t c = 0; c < D; ++c) acc[c] += p * vj[c];
                 }
                 double *o = out + ((size_t)bh * nrows + r) * D;
                 for (size_t c = 0; c < D; ++c) o[c] = acc[c] / z;
@@ -261,6 +272,7 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             free(qr);
             free(qx);
             free(s);
+            free(keys);
             free(acc);
         }
     }
