@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark: full 3D-RoPE attention throughput on B200.
+
+Headline metric: full 3D-RoPE attention TFLOP/s (4*N^2*d*heads per forward)
+and its fraction of the measured B200 dense bf16 peak, on the 81-frame
+480x832 clip: T'xH'xW' = 21x30x52 = 32,760 tokens, 12 heads x 128, B=1,
+RoPE split (44, 42, 42), seeded synthetic bf16 N(0,1) inputs.
+
+A step is one pass of the whole hot path: key RoPE pre-pass (rope3d_apply),
+angle table, and the fused Q-RoPE + attention kernel.  Inputs are resident
+in HBM before timing; Q, K, V and O together (403 MB) exceed the 126 MB L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs an independent replica of the workload (weak scaling, no collective on
+the data path) and rank 0 prints one JSON line.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HEAD_DIM = 128
+METRIC = "full 3D-RoPE attention TFLOP/s and % of B200 BF16 peak at 32,760 tokens"
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="c81f480")
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--no-extras", action="store_true", help="skip the secondary measurements")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "full_spatiotemporal_attention_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (its `source_hash` line matches)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_ncu.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                key, _, val = line[2:].partition(":")
+                vals[key.strip()] = val.strip().strip("`")
+    if vals.get("source_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons during the timed region."""
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8 or (self.uuid and parts[0] != self.uuid):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+
+def init_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        import torch
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def to_dev(bits, device):
+    import torch
+    return torch.from_numpy(bits).view(torch.bfloat16).to(device)
+
+
+def full_flops(w):
+    return 4.0 * w.N * w.N * HEAD_DIM * w.heads * w.batch
+
+
+def cpu_baseline(w, q, k, v, rows_per_head):
+    import oracle
+    import seeded_inputs as si
+    og = oracle.Grid(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    rows = si.sample_rows(w, rows_per_head)
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, og, rows=rows)
+    dt = time.perf_counter() - t0
+    flops = w.batch * w.heads * rows.size * 4.0 * w.N * HEAD_DIM
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{rows.size} seeded query rows x {w.batch * w.heads} heads of {w.name} "
+                      f"(N={w.N}); includes rotating all keys; {dt:.1f} s",
+            "seconds": round(dt, 3),
+            "extrapolated_full_forward_s": round(dt * w.N / rows.size, 1)}
+
+
+def timed_loop(fn, steps, warmup, world, device, marks=False):
+    """Run fn(i) warmup times untimed, then `steps` times between CUDA events.
+    fn may return a pair of events bracketing its dominant kernel."""
+    import torch
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    inner = []
+    start.record()
+    for i in range(steps):
+        ev = fn(i)
+        if ev is not None:
+            inner.append(ev)
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    total = start.elapsed_time(end)
+    inner_ms = [a.elapsed_time(b) for a, b in inner]
+    return total / steps, (sum(inner_ms) / len(inner_ms) if inner_ms else None)
+
+
+def bench_ours(args, rank, world, local):
+    import torch
+    import full_spatiotemporal_attention_b200 as va
+    import seeded_inputs as si
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = si.WORKLOADS[args.workload]
+    qb, kb, vb = si.qkv(w)
+    q, k, v = (to_dev(x, device) for x in (qb, kb, vb))
+    g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    kr = torch.empty_like(k)
+    o = torch.empty_like(q)
+    ws = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g, k_rotated=True),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        # key pre-pass, then (table + fused Q-RoPE attention) bracketed by events
+        va.rope3d_apply(k, g, out=kr)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        va.attn3d_full_fwd(q, kr, v, g, k_rotated=True, out=o, workspace=ws)
+        b.record(stream)
+        return a, b
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    step_ms, attn_ms = timed_loop(step, args.steps, args.warmup, world, device)
+    clocks = sampler.stop()
+    step_ms = max_over_ranks(step_ms, world, device)
+    attn_ms = max_over_ranks(attn_ms, world, device)
+
+    # key pre-pass alone (HBM-bound): bytes = read + write of K
+    def rope_only(i):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        va.rope3d_apply(k, g, out=kr)
+        b.record(stream)
+        return a, b
+    _, rope_ms = timed_loop(rope_only, max(args.steps, 10), 3, world, device)
+
+    flops = full_flops(w)
+    value = world * flops / (step_ms / 1e3) / 1e12
+    peak_tf, peak_gbs, peak_src = peaks()
+    achieved = flops / (attn_ms / 1e3) / 1e12
+    traffic = recorded_traffic("attn_fwd_kernel", w.name)
+
+    # end to end through the public API with host buffers
+    tensor_bytes = w.batch * w.heads * w.N * HEAD_DIM * 2
+    qh, kh, vh = (torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in (qb, kb, vb))
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd = (torch.empty_like(q) for _ in range(3))
+    ws_full = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g), dtype=torch.uint8,
+                          device=device)
+
+    def e2e_step(i):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        va.attn3d_full_fwd(qd, kd, vd, g, out=o, workspace=ws_full)
+        oh.copy_(o, non_blocking=True)
+    e2e_ms, _ = timed_loop(e2e_step, args.e2e_steps, 3, world, device)
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded splitmix64 + Box-Muller bf16 N(0,1))",
+        "config": {"workload": w.description, "grid": [w.T, w.H, w.W], "tokens": w.N,
+                   "heads": w.heads, "head_dim": HEAD_DIM, "batch": w.batch,
+                   "rope_split": list(w.dims), "theta": w.theta,
+                   "flops_per_step": flops, "global_batch": w.batch * world, "seq_len": w.N,
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)",
+                   "l2": "inputs exceed L2 (Q,K,V,O = 403 MB > 126 MB); no flush"},
+        "pct_of_peak": round(100.0 * value / world / peak_tf, 2),
+        "e2e": {"value": round(world * flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes},
+        "gpu_launches": 3 * args.steps,
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                     "traffic": traffic, "kernel": "attn_fwd_kernel",
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "kernel_ms": round(attn_ms, 4)},
+        "rope_prepass": {"kernel": "rope_apply_kernel", "ms": round(rope_ms, 4),
+                         "achieved_gbs": round(2 * tensor_bytes / (rope_ms / 1e3) / 1e9, 1),
+                         "peak_gbs": peak_gbs,
+                         "frac": round(2 * tensor_bytes / (rope_ms / 1e3) / 1e9 / peak_gbs, 4)},
+        "clocks": clocks,
+    }
+
+    if world == 1 and not args.no_extras:
+        line["extras"] = extras(va, device, stream, peak_tf, peak_gbs)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, qb, kb, vb, args.cpu_rows)
+    return line
+
+
+def extras(va, device, stream, peak_tf, peak_gbs):
+    """Secondary measurements: full vs factorised on the 720p clip (with the
+    temporal pass in GB/s) and joint video+text attention."""
+    import torch
+    import seeded_inputs as si
+    out = {}
+
+    def ev_pair(fn):
+        def run(i):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            return a, b
+        return run
+
+    w = si.WORKLOADS["c81f720"]
+    q, k, v = (to_dev(x, device) for x in si.qkv(w))
+    g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    kr = va.rope3d_apply(k, g)
+    o = torch.empty_like(q)
+    o2 = torch.empty_like(q)
+    ws = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g, k_rotated=True),
+                     dtype=torch.uint8, device=device)
+    _, full_ms = timed_loop(ev_pair(lambda: va.attn3d_full_fwd(q, kr, v, g, k_rotated=True, out=o,
+                                                               workspace=ws)), 3, 2, 1, device)
+    _, sp_ms = timed_loop(ev_pair(lambda: va.attn_factorized_fwd(
+        q, kr, v, g, temporal=False, k_rotated=True, out_spatial=o, workspace=ws)), 10, 3, 1, device)
+    _, tp_ms = timed_loop(ev_pair(lambda: va.attn_factorized_fwd(
+        q, kr, v, g, spatial=False, k_rotated=True, out_temporal=o2, workspace=ws)), 10, 3, 1, device)
+    hw = w.H * w.W
+    f_full = 4.0 * w.N ** 2 * HEAD_DIM * w.heads
+    f_sp = 4.0 * HEAD_DIM * w.heads * w.T * hw * hw
+    tbytes = 4 * w.heads * w.N * HEAD_DIM * 2
+    out["c81f720"] = {
+        "tokens": w.N, "heads": w.heads,
+        "full_ms": round(full_ms, 3), "full_tflops": round(f_full / full_ms / 1e9, 1),
+        "spatial_ms": round(sp_ms, 4), "spatial_tflops": round(f_sp / sp_ms / 1e9, 1),
+        "temporal_ms": round(tp_ms, 4), "temporal_gbs": round(tbytes / tp_ms / 1e6, 1),
+        "temporal_frac_hbm": round(tbytes / tp_ms / 1e6 / peak_gbs, 4),
+        "full_over_factorised_time": round(full_ms / (sp_ms + tp_ms), 2),
+        "full_over_factorised_flops": round(f_full / (f_sp + 4.0 * HEAD_DIM * w.heads * hw * w.T ** 2), 2),
+    }
+    del q, k, v, kr, o, o2, ws
+    torch.cuda.empty_cache()
+
+    w = si.WORKLOADS["joint720"]
+    q, k, v = (to_dev(x, device) for x in si.qkv(w))
+    g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    kr = va.rope3d_apply(k, g)
+    o = torch.empty_like(q)
+    ws = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g, k_rotated=True),
+                     dtype=torch.uint8, device=device)
+    _, j_ms = timed_loop(ev_pair(lambda: va.attn3d_full_fwd(q, kr, v, g, k_rotated=True, out=o,
+                                                            workspace=ws)), 3, 2, 1, device)
+    f_j = 4.0 * w.N ** 2 * HEAD_DIM * w.heads
+    out["joint720"] = {"tokens": w.N, "heads": w.heads, "ms": round(j_ms, 3),
+                       "tflops": round(f_j / j_ms / 1e9, 1),
+                       "frac_of_peak": round(f_j / j_ms / 1e9 / peak_tf, 4)}
+    del q, k, v, kr, o, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores: each step computes a
+    bounded sample of query rows of the same workload."""
+    import oracle
+    import seeded_inputs as si
+    w = si.WORKLOADS[args.workload]
+    q, k, v = si.qkv(w)
+    og = oracle.Grid(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    rows = si.sample_rows(w, 16)
+    flops = w.batch * w.heads * rows.size * 4.0 * w.N * HEAD_DIM
+    for _ in range(args.warmup):
+        oracle.attention(q, k, v, og, rows=rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attention(q, k, v, og, rows=rows)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = flops / dt / 1e12
+    sample = (f"{rows.size} seeded query rows x {w.batch * w.heads} heads of {w.name} per step "
+              f"(N={w.N}), all keys rotated each step")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.description, "tokens": w.N, "heads": w.heads},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3:
+        sys.exit("--warmup must be >= 3")
+    if args.impl == "reference":
+        # the oracle runs on rank 0 only; other ranks leave without work
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank == 0:
+            print(json.dumps(bench_reference(args, rank, world)), flush=True)
+        return
+    rank, world, local = init_dist(args)
+    line = bench_ours(args, rank, world, local)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

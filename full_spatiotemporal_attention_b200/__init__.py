@@ -1,0 +1,228 @@
+"""B200-native 3D-RoPE video self-attention: thin Python binding of libva3d.so.
+
+Every step of the hot path runs in the library's sm_100a kernels; this module
+only checks tensor properties and passes pointers, sizes and the current CUDA
+stream to the C ABI declared in ``include/va3d.h``.  There is no fallback: if
+the library is missing or a tensor is not a contiguous bf16 CUDA tensor of
+shape [B, heads, N, 128], the call raises.
+
+Entry points (same names as the C ABI):
+
+* ``rope3d_apply(x, grid)``                 3D RoPE of a [B, heads, N, 128] tensor
+* ``attn3d_full_fwd(q, k, v, grid)``        full 3D (or joint video+text) attention
+* ``attn_factorized_fwd(q, k, v, grid)``    spatial and temporal passes
+* ``grid_from_video(frames, height, width)``  token grid of a clip
+* ``workspace_bytes(...)``, ``device_error()``
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libva3d.so")
+
+VA3D_OK = 0
+VA3D_K_ROTATED = 1
+HEAD_DIM = 128
+
+SYMBOLS = ("va3d_status_string", "va3d_version", "va3d_grid_from_video",
+           "va3d_workspace_bytes", "rope3d_apply", "attn3d_full_fwd",
+           "attn_factorized_fwd", "va3d_device_error")
+
+
+class VA3DError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {status} ({_status_string(status)})")
+
+
+class Grid(ctypes.Structure):
+    """va3d_grid_t: post-patch grid T', H', W', appended text tokens, RoPE split, theta."""
+    _fields_ = [("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("n_text", ctypes.c_int),
+                ("d_t", ctypes.c_int), ("d_h", ctypes.c_int), ("d_w", ctypes.c_int),
+                ("theta", ctypes.c_double)]
+
+    @classmethod
+    def make(cls, T, H, W, n_text=0, dims=(44, 42, 42), theta=10000.0):
+        return cls(T, H, W, n_text, dims[0], dims[1], dims[2], theta)
+
+    @property
+    def n_video(self):
+        return self.T * self.H * self.W
+
+    @property
+    def N(self):
+        return self.n_video + self.n_text
+
+    def __repr__(self):
+        return (f"Grid(T={self.T}, H={self.H}, W={self.W}, n_text={self.n_text}, "
+                f"dims=({self.d_t}, {self.d_h}, {self.d_w}), theta={self.theta})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m full_spatiotemporal_attention_b200.build` "
+            "or __graft_entry__.build() (nvcc with sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, u, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t, ctypes.c_float
+    gp = ctypes.POINTER(Grid)
+    lib.va3d_status_string.argtypes = [i]
+    lib.va3d_status_string.restype = ctypes.c_char_p
+    lib.va3d_version.restype = i
+    lib.va3d_grid_from_video.argtypes = [i, i, i, i, i, i, i, gp]
+    lib.va3d_workspace_bytes.argtypes = [i, i, i, i, gp, u]
+    lib.va3d_workspace_bytes.restype = sz
+    lib.rope3d_apply.argtypes = [vp, vp, i, i, i, i, gp, vp]
+    lib.attn3d_full_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp, sz, vp]
+    lib.attn_factorized_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp, sz, vp]
+    lib.va3d_device_error.argtypes = [i]
+    return lib
+
+
+lib = _load()
+
+
+def _status_string(status):
+    return lib.va3d_status_string(int(status)).decode()
+
+
+def version():
+    return lib.va3d_version()
+
+
+def grid_from_video(frames, height, width, dims=(44, 42, 42), n_text=0):
+    """Token grid of a clip: T' = 1 + (frames-1)/4, H' = height/16, W' = width/16."""
+    g = Grid()
+    rc = lib.va3d_grid_from_video(frames, height, width, dims[0], dims[1], dims[2], n_text,
+                                  ctypes.byref(g))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_grid_from_video", rc)
+    return g
+
+
+def workspace_bytes(B, heads, N, grid, k_rotated=False):
+    return int(lib.va3d_workspace_bytes(B, heads, N, HEAD_DIM, ctypes.byref(grid),
+                                        VA3D_K_ROTATED if k_rotated else 0))
+
+
+# ---------------------------------------------------------------- tensors
+
+def _torch():
+    import torch
+    return torch
+
+
+def _check(t, name, shape=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.dim() != 4 or t.shape[-1] != HEAD_DIM:
+        raise ValueError(f"{name} must be [B, heads, N, {HEAD_DIM}], got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _stream(t):
+    return ctypes.c_void_p(_torch().cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _workspace(q, grid, k_rotated, workspace):
+    B, H, N, _ = q.shape
+    need = workspace_bytes(B, H, N, grid, k_rotated)
+    if workspace is None:
+        workspace = _torch().empty(max(need, 256), dtype=_torch().uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace holds {workspace.numel()} bytes, needs {need}")
+    return workspace
+
+
+def rope3d_apply(x, grid, out=None):
+    """3D RoPE of x [B, heads, N, 128] (bf16, CUDA); out may be x (in place)."""
+    _check(x, "x")
+    if out is None:
+        out = _torch().empty_like(x)
+    _check(out, "out", x.shape)
+    B, H, N, D = x.shape
+    rc = lib.rope3d_apply(_ptr(x), _ptr(out), B, H, N, D, ctypes.byref(grid), _stream(x))
+    if rc != VA3D_OK:
+        raise VA3DError("rope3d_apply", rc)
+    return out
+
+
+def attn3d_full_fwd(q, k, v, grid, *, scale=None, return_lse=False, k_rotated=False,
+                    out=None, lse=None, workspace=None):
+    """Full 3D attention (joint video+text when grid.n_text > 0).
+
+    Returns o [B, heads, N, 128] bf16 (and lse [B, heads, N] fp32 if asked)."""
+    torch = _torch()
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    B, H, N, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N)
+                            or not lse.is_contiguous() or not lse.is_cuda):
+        raise ValueError("lse must be a contiguous CUDA float32 [B, heads, N] tensor")
+    ws = _workspace(q, grid, k_rotated, workspace)
+    rc = lib.attn3d_full_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
+                             ctypes.byref(grid), float(scale or 0.0),
+                             VA3D_K_ROTATED if k_rotated else 0, _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(q))
+    if rc != VA3D_OK:
+        raise VA3DError("attn3d_full_fwd", rc)
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
+def attn_factorized_fwd(q, k, v, grid, *, spatial=True, temporal=True, scale=None,
+                        k_rotated=False, out_spatial=None, out_temporal=None, workspace=None):
+    """Factorised attention: (o_spatial, o_temporal); a skipped pass returns None."""
+    torch = _torch()
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    B, H, N, D = q.shape
+    if spatial and out_spatial is None:
+        out_spatial = torch.empty_like(q)
+    if temporal and out_temporal is None:
+        out_temporal = torch.empty_like(q)
+    if not spatial:
+        out_spatial = None
+    if not temporal:
+        out_temporal = None
+    for t, nm in ((out_spatial, "out_spatial"), (out_temporal, "out_temporal")):
+        if t is not None:
+            _check(t, nm, q.shape)
+    ws = _workspace(q, grid, k_rotated, workspace)
+    rc = lib.attn_factorized_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out_spatial),
+                                 _ptr(out_temporal), B, H, N, D, ctypes.byref(grid),
+                                 float(scale or 0.0), VA3D_K_ROTATED if k_rotated else 0,
+                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(q))
+    if rc != VA3D_OK:
+        raise VA3DError("attn_factorized_fwd", rc)
+    return out_spatial, out_temporal
+
+
+def device_error(reset=True):
+    """Watchdog code recorded on the current device (0 = none); synchronises."""
+    rc = lib.va3d_device_error(1 if reset else 0)
+    if rc < 0:
+        raise VA3DError("va3d_device_error", rc)
+    return rc

@@ -1,0 +1,408 @@
+// Flash-style attention forward on B200 tensor cores (tcgen05 + TMEM + TMA).
+//
+//   O = softmax(scale * Q~ K~^T) V over the keys of the query's segment,
+//
+// where Q~ is Q turned by 3D RoPE inside the kernel (right after its tile
+// lands in shared memory) and K~ is the pre-rotated key tensor.  Segments:
+// full 3D attention and joint video+text attention use one segment of N
+// tokens (handbook "How attention sees time": every token together); the
+// spatial pass of factorised attention uses T' segments of H'W' tokens (one
+// per frame).  The score matrix is never materialised (online softmax).
+//
+// CTA = one (batch*head, segment, 256 query rows) work tile, one CTA per SM:
+//   warps 0-3   softmax group 0: rows of query tile 0 (thread = TMEM lane = row)
+//   warps 4-7   softmax group 1: rows of query tile 1
+//   warp  8     tcgen05.mma issuer (one thread) and TMEM allocator
+//   warp  9     TMA loader (one thread)
+// TMEM (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1, 128 columns each;
+// P (bf16 pairs) overwrites the first 64 columns of its S.  The MMA issuer
+// ping-pongs the two query tiles so that one tile's softmax overlaps the
+// other tile's QK^T and PV products.  Q, K, V tiles are 128 rows x 128 bf16,
+// loaded by TMA as two 64-column boxes with the 128-byte swizzle.
+#pragma once
+
+#include "ptx.cuh"
+#include "rope.cuh"
+
+namespace va3d {
+namespace fa {
+
+constexpr int BM = 128;                    // query rows per tile
+constexpr int BN = 128;                    // keys per tile
+constexpr int HD = 128;                    // head dim
+constexpr int kStages = 2;                 // K and V ring depth
+constexpr int kThreads = 320;
+constexpr int kTileBytes = BM * HD * 2;    // 32 KB
+constexpr int kHalfBytes = kTileBytes / 2; // one 64-column box: 128 rows x 128 B
+
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + 2 * kTileBytes;
+constexpr int OFF_V = OFF_K + kStages * kTileBytes;
+constexpr int OFF_BAR = OFF_V + kStages * kTileBytes;
+
+enum Bar {
+    B_QFULL = 0,
+    B_QREADY0, B_QREADY1,
+    B_KFULL0, B_KFULL1,
+    B_KEMPTY0, B_KEMPTY1,
+    B_VFULL0, B_VFULL1,
+    B_VEMPTY0, B_VEMPTY1,
+    B_SFULL0, B_SFULL1,
+    B_PFULL0, B_PFULL1,
+    B_OFULL,
+    B_DRAIN,
+    NUM_BARS
+};
+
+constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
+constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
+constexpr int kSmemUsed = OFF_ABORT + 8;
+constexpr int kSmemBytes = kSmemUsed + 1024;   // slack to align the base to 1024 B
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 384;
+
+// Lazy rescaling: a row keeps its running maximum (log2 units) until a new
+// score exceeds it by more than this; P values then stay below 2^8.
+constexpr float kRescaleThreshold = 8.0f;
+
+struct AttnArgs {
+    int N;             // tokens per (batch, head) sequence
+    int seg_len;       // tokens per segment (N, or H'W' for the spatial pass)
+    int q_blocks;      // 256-row query blocks per segment
+    float scale_log2;  // softmax scale * log2(e)
+    int rope_q;        // 1: rotate Q tiles with the table
+    const float2 *rope_tab;
+    __nv_bfloat16 *o;
+    float *lse;        // may be null
+    RopeParams rp;
+};
+
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
+    // K-major, 128 B swizzle: 8-row groups 1024 B apart; the leading offset
+    // is unused for this layout (encoded as 16 B).
+    return smem_desc_sw128(saddr, 16, 1024);
+}
+
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr) {
+    // MN-major, 128 B swizzle: the two 64-element column blocks are one box
+    // (16 KB) apart; 8-row groups along K are 1024 B apart.
+    return smem_desc_sw128(saddr, kHalfBytes, 1024);
+}
+
+// Turn row `r` of a swizzled 128x128 Q tile in shared memory by 3D RoPE.
+__device__ __forceinline__ void rope_q_row(uint8_t *tile, int r, int n, const AttnArgs &a) {
+    const RopeParams &rp = a.rp;
+    if (n >= rp.n_video) return;   // text token or a padding row past N
+    const int t = n / rp.HW;
+    const int rem = n - t * rp.HW;
+    const int h = rem / rp.W;
+    const int w = rem - h * rp.W;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint4 *ptr = reinterpret_cast<uint4 *>(tile + half * kHalfBytes + r * 128 +
+                                                   ((c ^ (r & 7)) << 4));
+            uint4 v = *ptr;
+            const int p0 = half * 32 + c * 4;
+            v.x = rotate_pair(v.x, a.rope_tab[table_index(rp, p0 + 0, t, h, w)]);
+            v.y = rotate_pair(v.y, a.rope_tab[table_index(rp, p0 + 1, t, h, w)]);
+            v.z = rotate_pair(v.z, a.rope_tab[table_index(rp, p0 + 2, t, h, w)]);
+            v.w = rotate_pair(v.w, a.rope_tab[table_index(rp, p0 + 3, t, h, w)]);
+            *ptr = v;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const uint32_t sbase = smem_u32(smem);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
+    auto bar = [&](int i) -> uint32_t { return sbase + OFF_BAR + 8 * i; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int seg = blockIdx.x / a.q_blocks;
+    const int qb = blockIdx.x - seg * a.q_blocks;
+    const int seg_start = seg * a.seg_len;
+    const int seg_end = seg_start + a.seg_len;
+    const int q0 = seg_start + qb * (2 * BM);
+    const int n_kv = (a.seg_len + BN - 1) / BN;
+    const int kv_last_valid = a.seg_len - (n_kv - 1) * BN;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_QFULL), 1);
+        mbar_init(bar(B_QREADY0), BM);
+        mbar_init(bar(B_QREADY1), BM);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar(B_KFULL0 + s), 1);
+            mbar_init(bar(B_KEMPTY0 + s), 1);
+            mbar_init(bar(B_VFULL0 + s), 1);
+            mbar_init(bar(B_VEMPTY0 + s), 1);
+        }
+        mbar_init(bar(B_SFULL0), 1);
+        mbar_init(bar(B_SFULL1), 1);
+        mbar_init(bar(B_PFULL0), BM);
+        mbar_init(bar(B_PFULL1), BM);
+        mbar_init(bar(B_OFULL), 1);
+        mbar_init(bar(B_DRAIN), 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+        fence_proxy_async_smem();
+    }
+    if (warp == 8) tmem_alloc(sbase + OFF_TMEM_SLOT, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_TMEM_SLOT);
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ loader
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(bar(B_QFULL), 2 * kTileBytes);
+            for (int i = 0; i < 2; ++i)
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_3d(sbase + OFF_Q + i * kTileBytes + hf * kHalfBytes, &tmQ,
+                                bar(B_QFULL), hf * 64, q0 + i * BM, bh);
+            int last_k[kStages] = {-1, -1};   // last key tile issued into each stage
+            int last_v[kStages] = {-1, -1};
+            bool ok = true;
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                const int kv0 = seg_start + j * BN;
+                if (j >= kStages &&
+                    !(ok = mbar_wait(bar(B_KEMPTY0 + s), ph ^ 1, abort_flag, VA3D_DEVERR_TIMEOUT_LOAD)))
+                    break;
+                mbar_arrive_expect_tx(bar(B_KFULL0 + s), kTileBytes);
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_3d(sbase + OFF_K + s * kTileBytes + hf * kHalfBytes, &tmK,
+                                bar(B_KFULL0 + s), hf * 64, kv0, bh);
+                last_k[s] = j;
+                if (j >= kStages &&
+                    !(ok = mbar_wait(bar(B_VEMPTY0 + s), ph ^ 1, abort_flag, VA3D_DEVERR_TIMEOUT_LOAD)))
+                    break;
+                mbar_arrive_expect_tx(bar(B_VFULL0 + s), kTileBytes);
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_3d(sbase + OFF_V + s * kTileBytes + hf * kHalfBytes, &tmV,
+                                bar(B_VFULL0 + s), hf * 64, kv0, bh);
+                last_v[s] = j;
+            }
+            if (ok) {
+                // Producer tail: wait until the last tile of each stage has been
+                // released, so no barrier arrival can land after the CTA exits.
+                for (int s = 0; s < kStages && ok; ++s) {
+                    if (last_k[s] >= 0)
+                        ok = mbar_wait(bar(B_KEMPTY0 + s), (last_k[s] >> 1) & 1, abort_flag,
+                                       VA3D_DEVERR_TIMEOUT_LOAD);
+                    if (ok && last_v[s] >= 0)
+                        ok = mbar_wait(bar(B_VEMPTY0 + s), (last_v[s] >> 1) & 1, abort_flag,
+                                       VA3D_DEVERR_TIMEOUT_LOAD);
+                }
+            }
+            if (!ok) {
+                // Let the copies already in flight land before the CTA exits.
+                mbar_wait_drain(bar(B_QFULL), 0);
+                for (int s = 0; s < kStages; ++s) {
+                    if (last_k[s] >= 0) mbar_wait_drain(bar(B_KFULL0 + s), (last_k[s] >> 1) & 1);
+                    if (last_v[s] >= 0) mbar_wait_drain(bar(B_VFULL0 + s), (last_v[s] >> 1) & 1);
+                }
+            }
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, 0);
+            constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, 1);
+
+            auto issue_s = [&](int i, int s) {
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                    mma_ss(tmem + COL_S0 + i * (COL_S1 - COL_S0), desc_kmajor(sbase + OFF_Q + i * kTileBytes + off),
+                           desc_kmajor(sbase + OFF_K + s * kTileBytes + off), kIdescQK, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int i, int s, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    mma_ts(tmem + COL_O0 + i * (COL_O1 - COL_O0), tmem + COL_S0 + i * (COL_S1 - COL_S0) + kk * 8,
+                           desc_mnmajor(sbase + OFF_V + s * kTileBytes + kk * 2048), kIdescPV,
+                           (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+
+            bool ok = mbar_wait(bar(B_QREADY0), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA) &&
+                      mbar_wait(bar(B_QREADY1), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA) &&
+                      mbar_wait(bar(B_KFULL0), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                mma_commit(bar(B_SFULL0));
+                issue_s(1, 0);
+                mma_commit(bar(B_SFULL1));
+                mma_commit(bar(B_KEMPTY0));
+            }
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int s = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                const bool more = j + 1 < n_kv;
+                const int s2 = (j + 1) & 1;
+                const uint32_t ph2 = ((j + 1) >> 1) & 1;
+                ok = mbar_wait(bar(B_VFULL0 + s), ph, abort_flag, VA3D_DEVERR_TIMEOUT_MMA) &&
+                     mbar_wait(bar(B_PFULL0), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(0, s, j > 0);
+                if (more) {
+                    ok = mbar_wait(bar(B_KFULL0 + s2), ph2, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(0, s2);
+                    mma_commit(bar(B_SFULL0));
+                }
+                ok = mbar_wait(bar(B_PFULL1), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(1, s, j > 0);
+                mma_commit(bar(B_VEMPTY0 + s));
+                if (more) {
+                    issue_s(1, s2);
+                    mma_commit(bar(B_SFULL1));
+                    mma_commit(bar(B_KEMPTY0 + s2));
+                }
+            }
+            if (ok) {
+                mma_commit(bar(B_OFULL));
+            } else {
+                // Wait for the products already issued before TMEM is freed.
+                mma_commit(bar(B_DRAIN));
+                mbar_wait_drain(bar(B_DRAIN), 0);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- softmax
+        const int g = warp >> 2;                  // query tile of this group
+        const int r = ((warp & 3) << 5) + lane;   // row in the tile = TMEM lane
+        const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) << 5) << 16;
+        const uint32_t taS = tmem + lane_addr + (g ? COL_S1 : COL_S0);
+        const uint32_t taO = tmem + lane_addr + (g ? COL_O1 : COL_O0);
+        const int n = q0 + g * BM + r;            // token index of this row
+
+        bool ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QFULL), 0, abort_flag,
+                                                    VA3D_DEVERR_TIMEOUT_SOFTMAX));
+        if (ok) {
+            if (a.rope_q) rope_q_row(smem + OFF_Q + g * kTileBytes, r, n, a);
+            fence_proxy_async_smem();
+            mbar_arrive(bar(g ? B_QREADY1 : B_QREADY0));
+        }
+
+        float m_ref = -INFINITY;   // running row maximum, log2 units (scaled)
+        float l = 0.0f;            // running row sum of exp2
+        for (int j = 0; j < n_kv && ok; ++j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(g ? B_SFULL1 : B_SFULL0), j & 1,
+                                                   abort_flag, VA3D_DEVERR_TIMEOUT_SOFTMAX));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sr[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_ld32(taS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+            float *s = reinterpret_cast<float *>(sr);
+            if (j == n_kv - 1 && kv_last_valid < BN) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (c >= kv_last_valid) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+            const float m_new = fmaxf(m_ref, mx * a.scale_log2);
+            float alpha = 1.0f;
+            const bool bump = m_new - m_ref > kRescaleThreshold;
+            if (bump) {
+                alpha = ex2(m_ref - m_new);
+                m_ref = m_new;
+            }
+            const float neg_m = -m_ref;
+            float rowsum = 0.0f;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = ex2(fmaf(s[64 * hf + 2 * c], a.scale_log2, neg_m));
+                    const float p1 = ex2(fmaf(s[64 * hf + 2 * c + 1], a.scale_log2, neg_m));
+                    rowsum += p0 + p1;
+                    pk[c] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(taS + 32 * hf, pk);
+            }
+            if (j > 0 && __any_sync(0xffffffffu, bump)) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(taO + 32 * c, ov);
+                    tmem_wait_ld();
+                    reg_fence32(ov);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                    tmem_st32(taO + 32 * c, ov);
+                }
+            }
+            l = l * alpha + rowsum;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(g ? B_PFULL1 : B_PFULL0));
+        }
+
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), 0, abort_flag,
+                                                       VA3D_DEVERR_TIMEOUT_SOFTMAX));
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = 1.0f / l;
+            const bool valid = n < seg_end;
+            uint4 *dst = reinterpret_cast<uint4 *>(a.o + (static_cast<size_t>(bh) * a.N + n) * HD);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t ov[32];
+                tmem_ld32(taO + 32 * c, ov);
+                tmem_wait_ld();
+                reg_fence32(ov);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l,
+                                        __uint_as_float(ov[2 * e + 1]) * inv_l);
+                if (valid) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
+                                                    pk[4 * e + 3]);
+                }
+            }
+            if (a.lse != nullptr && valid)
+                a.lse[static_cast<size_t>(bh) * a.N + n] = (m_ref + log2f(l)) * 0.69314718055994531f;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 8) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace fa
+}  // namespace va3d

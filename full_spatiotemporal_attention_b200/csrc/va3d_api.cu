@@ -1,0 +1,358 @@
+// C ABI of libva3d.so: argument checks, tensor-map construction and kernel
+// launches.  The whole library is one translation unit (the kernels live in
+// the headers included below) so the device error word is shared by every
+// kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "va3d.h"
+#include "ptx.cuh"
+#include "rope.cuh"
+#include "attn_sm100.cuh"
+#include "attn_temporal.cuh"
+
+using namespace va3d;
+
+namespace {
+
+constexpr int kHeadDim = 128;
+constexpr double kLog2e = 1.4426950408889634;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int check_grid(const va3d_grid_t *g, int N, int head_dim) {
+    if (g == nullptr) return VA3D_ERR_INVALID;
+    if (g->T < 1 || g->H < 1 || g->W < 1 || g->n_text < 0) return VA3D_ERR_INVALID;
+    if (g->d_t < 0 || g->d_h < 0 || g->d_w < 0) return VA3D_ERR_INVALID;
+    if ((g->d_t | g->d_h | g->d_w) & 1) return VA3D_ERR_INVALID;
+    if (g->d_t + g->d_h + g->d_w != head_dim) return VA3D_ERR_INVALID;
+    if (!(g->theta > 0.0) || !std::isfinite(g->theta)) return VA3D_ERR_INVALID;
+    const long long nv = static_cast<long long>(g->T) * g->H * g->W;
+    if (nv + g->n_text != N) return VA3D_ERR_INVALID;
+    return VA3D_OK;
+}
+
+int check_sizes(int B, int heads, int N, int head_dim) {
+    if (B < 1 || heads < 1 || N < 1) return VA3D_ERR_INVALID;
+    if (head_dim != kHeadDim) return VA3D_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * heads > 65535) return VA3D_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * heads * N * kHeadDim * 2 > (1ll << 40)) return VA3D_ERR_UNSUPPORTED;
+    return VA3D_OK;
+}
+
+int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return VA3D_ERR_CUDA;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return VA3D_ERR_CUDA;
+    if (major != 10 || minor != 0) return VA3D_ERR_DEVICE;
+    return VA3D_OK;
+}
+
+long long table_entries(const va3d_grid_t *g) {
+    return static_cast<long long>(g->T) * (g->d_t / 2) + static_cast<long long>(g->H) * (g->d_h / 2) +
+           static_cast<long long>(g->W) * (g->d_w / 2);
+}
+
+size_t table_bytes(const va3d_grid_t *g) { return round_up(8 * table_entries(g), 256); }
+
+size_t tensor_bytes(int B, int heads, int N) {
+    return static_cast<size_t>(B) * heads * N * kHeadDim * 2;
+}
+
+RopeParams make_rope_params(const va3d_grid_t *g) {
+    RopeParams rp;
+    std::memset(&rp, 0, sizeof rp);
+    rp.T = g->T;
+    rp.H = g->H;
+    rp.W = g->W;
+    rp.HW = g->H * g->W;
+    rp.n_video = g->T * g->H * g->W;
+    rp.half_t = g->d_t / 2;
+    rp.half_h = g->d_h / 2;
+    rp.half_w = g->d_w / 2;
+    rp.pe_t = rp.half_t;
+    rp.pe_h = rp.half_t + rp.half_h;
+    rp.tab_h = g->T * rp.half_t;
+    rp.tab_w = rp.tab_h + g->H * rp.half_h;
+    rp.tab_entries = rp.tab_w + g->W * rp.half_w;
+    // inverse frequency of every pair: theta^(-2j/d) for index j in its axis range
+    const int dims[3] = {g->d_t, g->d_h, g->d_w};
+    int p = 0;
+    for (int ax = 0; ax < 3; ++ax)
+        for (int j = 0; j < dims[ax] / 2; ++j, ++p)
+            rp.inv_freq[p] = static_cast<float>(std::pow(g->theta, -2.0 * j / dims[ax]));
+    return rp;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// [BH, N, 128] bf16 viewed as a 3D tensor (dim, row, bh); boxes of
+// 64 columns x 128 rows with the 128-byte swizzle; rows past N read as zero.
+int make_map(CUtensorMap *map, const void *base, int N, int BH) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return VA3D_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(N),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2,
+                             static_cast<cuuint64_t>(N) * kHeadDim * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VA3D_OK : VA3D_ERR_CUDA;
+}
+
+int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? VA3D_OK : VA3D_ERR_CUDA;
+}
+
+int launch_table(float2 *tab, const RopeParams &rp, cudaStream_t st) {
+    if (rp.tab_entries == 0) return VA3D_OK;
+    const int threads = 256;
+    const int blocks = (rp.tab_entries + threads - 1) / threads;
+    rope_table_kernel<<<blocks, threads, 0, st>>>(tab, rp);
+    return launch_status();
+}
+
+int launch_rope(const void *x, void *y, int BH, int N, const RopeParams &rp, cudaStream_t st) {
+    const long long threads = static_cast<long long>(N) * 16;
+    const long long blocks = (threads + kRopeThreads - 1) / kRopeThreads;
+    rope_apply_kernel<<<static_cast<unsigned>(blocks), kRopeThreads, 0, st>>>(
+        static_cast<const uint4 *>(x), static_cast<uint4 *>(y), N, BH, rp);
+    return launch_status();
+}
+
+// Attention over segments of seg_len tokens (n_seg * seg_len == n_video or N).
+int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float *lse, int BH, int N,
+                int seg_len, int n_seg, const RopeParams &rp, const float2 *tab, float scale,
+                cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    int rc;
+    if ((rc = make_map(&mq, q, N, BH)) != VA3D_OK) return rc;
+    if ((rc = make_map(&mk, k_rot, N, BH)) != VA3D_OK) return rc;
+    if ((rc = make_map(&mv, v, N, BH)) != VA3D_OK) return rc;
+    fa::AttnArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.N = N;
+    a.seg_len = seg_len;
+    a.q_blocks = (seg_len + 2 * fa::BM - 1) / (2 * fa::BM);
+    a.scale_log2 = static_cast<float>(scale * kLog2e);
+    a.rope_q = 1;
+    a.rope_tab = tab;
+    a.o = static_cast<__nv_bfloat16 *>(o);
+    a.lse = lse;
+    a.rp = rp;
+    if (cudaFuncSetAttribute(fa::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::kSmemBytes) != cudaSuccess)
+        return VA3D_ERR_CUDA;
+    const long long gx = static_cast<long long>(n_seg) * a.q_blocks;
+    if (gx > 0x7fffffffll) return VA3D_ERR_UNSUPPORTED;
+    dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(BH));
+    fa::attn_fwd_kernel<<<grid, fa::kThreads, fa::kSmemBytes, st>>>(mq, mk, mv, a);
+    return launch_status();
+}
+
+template <int MAXT>
+int launch_temporal_t(const tp::TemporalArgs &a, cudaStream_t st) {
+    constexpr int smem = tp::Cfg<MAXT>::kSmemBytes;
+    if (cudaFuncSetAttribute(tp::temporal_kernel<MAXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+        return VA3D_ERR_CUDA;
+    const long long tasks = static_cast<long long>(a.BH) * a.HW;
+    const long long blocks = (tasks + tp::Cfg<MAXT>::kWarps - 1) / tp::Cfg<MAXT>::kWarps;
+    if (blocks > 0x7fffffffll) return VA3D_ERR_UNSUPPORTED;
+    tp::temporal_kernel<MAXT><<<static_cast<unsigned>(blocks), tp::Cfg<MAXT>::kWarps * 32, smem, st>>>(a);
+    return launch_status();
+}
+
+int launch_temporal(const void *q, const void *k_rot, const void *v, void *o, int BH, int N,
+                    const RopeParams &rp, const float2 *tab, float scale, cudaStream_t st) {
+    tp::TemporalArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.k = static_cast<const __nv_bfloat16 *>(k_rot);
+    a.v = static_cast<const __nv_bfloat16 *>(v);
+    a.o = static_cast<__nv_bfloat16 *>(o);
+    a.N = N;
+    a.T = rp.T;
+    a.HW = rp.HW;
+    a.BH = BH;
+    a.scale_log2 = static_cast<float>(scale * kLog2e);
+    a.rope_q = 1;
+    a.rope_tab = tab;
+    a.rp = rp;
+    if (rp.T <= 32) return launch_temporal_t<32>(a, st);
+    return launch_temporal_t<64>(a, st);
+}
+
+// Shared front half of the two attention entry points: checks, workspace
+// split, angle table and (unless the keys come rotated) the key pre-pass.
+struct Prepared {
+    RopeParams rp;
+    const float2 *tab;
+    const void *k_rot;
+    float scale;
+};
+
+int prepare(const void *q, const void *k, const void *v, int B, int heads, int N, int head_dim,
+            const va3d_grid_t *grid, float softmax_scale, unsigned flags, void *workspace,
+            size_t workspace_bytes, cudaStream_t st, Prepared *out) {
+    int rc;
+    if ((rc = check_sizes(B, heads, N, head_dim)) != VA3D_OK) return rc;
+    if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
+    if (q == nullptr || k == nullptr || v == nullptr) return VA3D_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return VA3D_ERR_ALIGNMENT;
+    if (flags & ~static_cast<unsigned>(VA3D_K_ROTATED)) return VA3D_ERR_INVALID;
+    const size_t need = va3d_workspace_bytes(B, heads, N, head_dim, grid, flags);
+    if (workspace == nullptr || workspace_bytes < need) return VA3D_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+
+    out->rp = make_rope_params(grid);
+    out->tab = static_cast<const float2 *>(workspace);
+    out->scale = softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(double(head_dim)));
+    if ((rc = launch_table(static_cast<float2 *>(workspace), out->rp, st)) != VA3D_OK) return rc;
+    if (flags & VA3D_K_ROTATED) {
+        out->k_rot = k;
+    } else {
+        void *kr = static_cast<uint8_t *>(workspace) + table_bytes(grid);
+        if ((rc = launch_rope(k, kr, B * heads, N, out->rp, st)) != VA3D_OK) return rc;
+        out->k_rot = kr;
+    }
+    return VA3D_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *va3d_status_string(int status) {
+    switch (status) {
+    case VA3D_OK: return "success";
+    case VA3D_ERR_INVALID: return "invalid argument (null pointer, size or grid)";
+    case VA3D_ERR_UNSUPPORTED: return "unsupported size (head_dim must be 128; see limits)";
+    case VA3D_ERR_ALIGNMENT: return "pointer not 16-byte aligned (workspace: 256-byte)";
+    case VA3D_ERR_WORKSPACE: return "workspace missing or too small";
+    case VA3D_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case VA3D_ERR_DEVICE: return "current device is not compute capability 10.0 (B200)";
+    default: return "unknown status";
+    }
+}
+
+int va3d_version(void) { return 100; }
+
+int va3d_grid_from_video(int frames, int height, int width, int d_t, int d_h, int d_w, int n_text,
+                         va3d_grid_t *out) {
+    if (out == nullptr || frames < 1 || height < 16 || width < 16 || n_text < 0) return VA3D_ERR_INVALID;
+    if ((frames - 1) % 4 != 0 || height % 16 != 0 || width % 16 != 0) return VA3D_ERR_INVALID;
+    va3d_grid_t g;
+    g.T = 1 + (frames - 1) / 4;
+    g.H = height / 16;
+    g.W = width / 16;
+    g.n_text = n_text;
+    g.d_t = d_t;
+    g.d_h = d_h;
+    g.d_w = d_w;
+    g.theta = 10000.0;
+    *out = g;
+    return VA3D_OK;
+}
+
+size_t va3d_workspace_bytes(int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
+                            unsigned flags) {
+    if (check_sizes(B, heads, N, head_dim) != VA3D_OK) return 0;
+    if (check_grid(grid, N, head_dim) != VA3D_OK) return 0;
+    size_t bytes = table_bytes(grid);
+    if (!(flags & VA3D_K_ROTATED)) bytes += tensor_bytes(B, heads, N);
+    return bytes;
+}
+
+int rope3d_apply(const va3d_bf16 *x, va3d_bf16 *y, int B, int heads, int N, int head_dim,
+                 const va3d_grid_t *grid, void *stream) {
+    int rc;
+    if ((rc = check_sizes(B, heads, N, head_dim)) != VA3D_OK) return rc;
+    if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
+    if (x == nullptr || y == nullptr) return VA3D_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(y)) return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    return launch_rope(x, y, B * heads, N, make_rope_params(grid), static_cast<cudaStream_t>(stream));
+}
+
+int attn3d_full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *o,
+                    float *lse, int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
+                    float softmax_scale, unsigned flags, void *workspace, size_t workspace_bytes,
+                    void *stream) {
+    if (o == nullptr) return VA3D_ERR_INVALID;
+    if (!aligned16(o) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return VA3D_ERR_ALIGNMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Prepared p;
+    int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
+                     workspace_bytes, st, &p);
+    if (rc != VA3D_OK) return rc;
+    return launch_attn(q, p.k_rot, v, o, lse, B * heads, N, N, 1, p.rp, p.tab, p.scale, st);
+}
+
+int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
+                        va3d_bf16 *o_spatial, va3d_bf16 *o_temporal, int B, int heads, int N,
+                        int head_dim, const va3d_grid_t *grid, float softmax_scale, unsigned flags,
+                        void *workspace, size_t workspace_bytes, void *stream) {
+    if (o_spatial == nullptr && o_temporal == nullptr) return VA3D_ERR_INVALID;
+    if ((o_spatial && !aligned16(o_spatial)) || (o_temporal && !aligned16(o_temporal)))
+        return VA3D_ERR_ALIGNMENT;
+    if (grid == nullptr) return VA3D_ERR_INVALID;
+    if (grid->n_text != 0) return VA3D_ERR_INVALID;
+    if (o_temporal != nullptr && grid->T > 64) return VA3D_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Prepared p;
+    int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
+                     workspace_bytes, st, &p);
+    if (rc != VA3D_OK) return rc;
+    if (o_spatial != nullptr) {
+        rc = launch_attn(q, p.k_rot, v, o_spatial, nullptr, B * heads, N, p.rp.HW, p.rp.T, p.rp,
+                         p.tab, p.scale, st);
+        if (rc != VA3D_OK) return rc;
+    }
+    if (o_temporal != nullptr)
+        rc = launch_temporal(q, p.k_rot, v, o_temporal, B * heads, N, p.rp, p.tab, p.scale, st);
+    return rc;
+}
+
+int va3d_device_error(int reset) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return VA3D_ERR_CUDA;
+    int value = 0;
+    if (cudaMemcpyFromSymbol(&value, va3d::g_device_error, sizeof value) != cudaSuccess)
+        return VA3D_ERR_CUDA;
+    if (reset) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(va3d::g_device_error, &zero, sizeof zero) != cudaSuccess)
+            return VA3D_ERR_CUDA;
+    }
+    return value;
+}
+
+}  // extern "C"

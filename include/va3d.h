@@ -1,0 +1,180 @@
+/*
+ * va3d: 3D-RoPE video self-attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libva3d.so.  Plain pointers and sizes only; no CUDA or framework
+ * types appear in the signatures (a CUDA stream is passed as void*).
+ *
+ * Operations and where they are defined:
+ *  - token grid: "A video model's architecture: spatiotemporal attention and
+ *    the 3D VAE" (anrans.github.io ai-infra-handbooks), section "The latents:
+ *    the extra time axis": T' = 1 + (T-1)/4, H' = H/8/2, W' = W/8/2;
+ *  - 3D RoPE: same page, section "Position: RoPE in three dimensions" (head
+ *    dim split into t, h and w ranges, each rotated by its coordinate), and
+ *    "CogVideoX Architecture ..." (aifetchly-blog) section 3, block-diagonal
+ *    R_3D(t, y, x);
+ *  - full, spatial and temporal attention: handbook page, section "How
+ *    attention sees time: factorised or full";
+ *  - joint video+text attention: "04 HunyuanVideo and Wan" (note.shouss.top)
+ *    sections 2.3-2.4, and the handbook's diffusers example (video tokens +
+ *    text tokens attended together in one sequence).
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are contiguous bf16 (bit patterns, va3d_bf16) of shape
+ *    [B, heads, N, head_dim], row-major, head_dim innermost.  Every pointer
+ *    must be 16-byte aligned.  head_dim must be 128.
+ *  - Token n of a sequence is a video token when n < T'H'W', with
+ *    t = n / (H'W'), h = (n / W') % H', w = n % W' (w fastest); tokens
+ *    n >= T'H'W' are text tokens, which carry no position (identity RoPE).
+ *    N must equal T'H'W' + n_text.
+ *  - RoPE: the head dim is split into ranges [0, d_t), [d_t, d_t+d_h),
+ *    [d_t+d_h, 128) turned by t, h and w; inside a range of width d the
+ *    adjacent pair (2j, 2j+1) turns by pos * theta^(-2j/d).
+ *  - Memory is owned by the caller.  No entry point allocates device memory;
+ *    scratch space is the caller's `workspace` (size from
+ *    va3d_workspace_bytes).  Device pointers must belong to the current
+ *    device.  Two calls that share a workspace must not overlap in time.
+ *  - Calls are asynchronous on `stream` (NULL = legacy default stream).  The
+ *    return value reports argument errors and launch errors only; device-side
+ *    faults surface at the caller's next synchronisation.  A device-side
+ *    watchdog (every wait in the kernels is bounded) records a code that
+ *    va3d_device_error() returns.
+ *  - Entry points are thread-safe: they keep no mutable host state.
+ */
+#ifndef VA3D_H
+#define VA3D_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t va3d_bf16;   /* bf16 bit pattern */
+
+/* Post-patch token grid and RoPE split. */
+typedef struct va3d_grid {
+    int T, H, W;        /* latent grid after patchify: T', H', W' (each >= 1) */
+    int n_text;         /* text tokens appended after the video tokens (>= 0) */
+    int d_t, d_h, d_w;  /* RoPE ranges; each even and >= 0, sum == head_dim */
+    double theta;       /* RoPE base (> 0), 10000 for the models on the pages */
+} va3d_grid_t;
+
+/* Status codes (0 = success, negative = error). */
+enum {
+    VA3D_OK = 0,
+    VA3D_ERR_INVALID = -1,      /* null pointer, non-positive size, inconsistent grid */
+    VA3D_ERR_UNSUPPORTED = -2,  /* head_dim != 128, or a size the kernels do not cover */
+    VA3D_ERR_ALIGNMENT = -3,    /* a pointer is not 16-byte aligned */
+    VA3D_ERR_WORKSPACE = -4,    /* workspace missing or smaller than va3d_workspace_bytes */
+    VA3D_ERR_CUDA = -5,         /* a CUDA runtime or driver call failed */
+    VA3D_ERR_DEVICE = -6        /* current device is not compute capability 10.0 */
+};
+
+/* Flags for the attention entry points. */
+enum {
+    VA3D_K_ROTATED = 1          /* `k` already holds RoPE-rotated keys (no key pre-pass) */
+};
+
+/* Device-side watchdog codes returned by va3d_device_error(). */
+enum {
+    VA3D_DEVERR_NONE = 0,
+    VA3D_DEVERR_TIMEOUT_LOAD = 1,     /* a wait in the tile-loading role timed out */
+    VA3D_DEVERR_TIMEOUT_MMA = 2,      /* a wait in the MMA-issuing role timed out */
+    VA3D_DEVERR_TIMEOUT_SOFTMAX = 3   /* a wait in the softmax role timed out */
+};
+
+/* Human-readable text of a status code; never NULL. */
+const char *va3d_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int va3d_version(void);
+
+/*
+ * Token grid of a clip (handbook, "The latents: the extra time axis"):
+ * T' = 1 + (frames - 1)/4, H' = height/16, W' = width/16.  Requires
+ * frames = 4k + 1 >= 1 and height, width positive multiples of 16 (the
+ * causal VAE's 4k+1 frame rule, 8x spatial compression, 2x2 patches);
+ * otherwise returns VA3D_ERR_INVALID and leaves *out untouched.  The RoPE
+ * split and text length are copied into *out; theta is set to 10000.
+ * Host-only; needs no device.
+ */
+int va3d_grid_from_video(int frames, int height, int width, int d_t, int d_h, int d_w,
+                         int n_text, va3d_grid_t *out);
+
+/*
+ * Bytes of scratch space attn3d_full_fwd / attn_factorized_fwd need for
+ * these arguments: a cos/sin table of the grid's rotation angles
+ * (8 * (T'*d_t/2 + H'*d_h/2 + W'*d_w/2) bytes, rounded up to 256) plus,
+ * unless flags has VA3D_K_ROTATED, the rotated keys (B*heads*N*head_dim*2
+ * bytes).  Returns 0 for invalid arguments.  Host-only.
+ */
+size_t va3d_workspace_bytes(int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
+                            unsigned flags);
+
+/*
+ * 3D RoPE (handbook "Position: RoPE in three dimensions"; CogVideoX guide
+ * section 3, R_3D block-diagonal matrix): y = R_3D(t, h, w) x for every
+ * video token, y = x for text tokens.
+ *   x, y    device, [B, heads, N, head_dim] bf16; x == y (in place) is allowed,
+ *           other overlap is not.  Output rounded to bf16 (nearest even);
+ *           angles are computed in fp32 from fp64 inverse frequencies.
+ *   stream  cudaStream_t or NULL.
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _ALIGNMENT, _DEVICE, _CUDA.
+ */
+int rope3d_apply(const va3d_bf16 *x, va3d_bf16 *y, int B, int heads, int N, int head_dim,
+                 const va3d_grid_t *grid, void *stream);
+
+/*
+ * Full 3D attention (handbook "How attention sees time": every token attends
+ * to every token); with grid->n_text > 0 this is joint video+text attention
+ * (HunyuanVideo/CogVideoX joint attention over the concatenated sequence,
+ * text appended after the video tokens, no mask):
+ *   o = softmax(scale * RoPE(q) RoPE(k)^T) v,   lse = log-sum-exp of the row.
+ *   q, k, v   device, [B, heads, N, head_dim] bf16, read only.  When flags
+ *             has VA3D_K_ROTATED, k must already be rotated (e.g. by
+ *             rope3d_apply) and q is still rotated inside the kernel.
+ *   o         device, [B, heads, N, head_dim] bf16, written; must not overlap
+ *             the inputs or the workspace.
+ *   lse       device fp32 [B, heads, N] (natural log), or NULL.
+ *   softmax_scale  <= 0 selects 1/sqrt(head_dim).
+ *   workspace, workspace_bytes  device scratch of at least
+ *             va3d_workspace_bytes(B, heads, N, head_dim, grid, flags) bytes,
+ *             256-byte aligned; contents are overwritten.
+ * Accumulation is fp32; P is rounded to bf16 before the PV product; o is
+ * rounded to bf16 (nearest even).
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _ALIGNMENT, _WORKSPACE, _DEVICE, _CUDA.
+ */
+int attn3d_full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
+                    va3d_bf16 *o, float *lse, int B, int heads, int N, int head_dim,
+                    const va3d_grid_t *grid, float softmax_scale, unsigned flags,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Factorised spatiotemporal attention (handbook "How attention sees time":
+ * spatial attention inside each frame, T' sequences of H'W' tokens, then
+ * temporal attention at each spatial position, H'W' sequences of T' tokens).
+ * Both passes read the same rotated q, k and v and write separate outputs:
+ *   o_spatial  [B, heads, N, head_dim]: token attends to tokens with equal t;
+ *   o_temporal [B, heads, N, head_dim]: token attends to tokens with equal (h, w).
+ * Either output may be NULL to skip that pass.  grid->n_text must be 0.  The
+ * temporal pass needs T' <= 64.  Other arguments as in attn3d_full_fwd.
+ * Errors: as attn3d_full_fwd.
+ */
+int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
+                        va3d_bf16 *o_spatial, va3d_bf16 *o_temporal, int B, int heads, int N,
+                        int head_dim, const va3d_grid_t *grid, float softmax_scale,
+                        unsigned flags, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Last device-side watchdog code recorded on the current device
+ * (VA3D_DEVERR_*; 0 = none).  Synchronises the device.  With reset != 0 the
+ * word is cleared afterwards.  Returns VA3D_ERR_CUDA if it cannot be read.
+ */
+int va3d_device_error(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VA3D_H */

@@ -1,0 +1,198 @@
+"""Parity of the sm_100a kernels (through the C ABI) with the fp64 oracle.
+
+Bar (per BASELINE's stated tolerance for bf16 outputs with fp32
+accumulation): max-abs error <= 1.5e-2 and mean-abs error <= 2e-3; in
+addition the relative L2 error must stay <= 2e-2, which is the meaningful
+gate at large N where outputs are small.  Small workloads compare every
+row; the full-size workloads (the configuration the bench times) compare
+512 seeded query rows per head, always including the first and last rows,
+tile and frame boundaries and, for joint attention, at least 64 text rows.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import seeded_inputs as si
+from conftest import bf16_bits_to_f64
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+MAX_ABS, MEAN_ABS, REL_L2 = 1.5e-2, 2e-3, 2e-2
+
+
+@pytest.fixture(scope="module")
+def va():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from full_spatiotemporal_attention_b200 import build
+    build.build()
+    import full_spatiotemporal_attention_b200 as va
+    assert torch.cuda.get_device_capability() == (10, 0), "kernels target sm_100a (B200)"
+    return va
+
+
+def dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).cuda()
+
+
+def host(t):
+    return bf16_bits_to_f64(t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+def vgrid(va, w):
+    return va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+
+
+def ogrid(w):
+    return oracle.Grid(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+
+
+def check(got, ref, label):
+    err = np.abs(got - ref)
+    max_abs, mean_abs = float(err.max()), float(err.mean())
+    rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    assert np.isfinite(got).all(), f"{label}: non-finite output"
+    assert max_abs <= MAX_ABS and mean_abs <= MEAN_ABS and rel <= REL_L2, (
+        f"{label}: max_abs={max_abs:.3e} mean_abs={mean_abs:.3e} rel_l2={rel:.3e}")
+    return max_abs, mean_abs, rel
+
+
+def custom(name, T, H, W, heads=2, n_text=0, dims=(44, 42, 42), batch=1, seed=7):
+    return si.Workload(name, T, H, W, heads, dims, n_text=n_text, batch=batch, seed=seed)
+
+
+SMALL = [si.WORKLOADS["tiny"], si.WORKLOADS["c17f480"],
+         custom("n1", 1, 1, 1), custom("n127", 1, 1, 127), custom("n129", 1, 3, 43),
+         custom("n257", 1, 1, 257, dims=(16, 56, 56)), custom("odd", 3, 5, 17, heads=3),
+         custom("batch2", 2, 7, 9, heads=2, batch=2),
+         custom("joint_small", 2, 6, 10, heads=2, n_text=37, dims=(16, 56, 56)),
+         custom("text1", 1, 4, 4, n_text=1), custom("mostly_text", 1, 2, 2, n_text=300)]
+
+FACTORISED_SMALL = [si.WORKLOADS["tiny"], si.WORKLOADS["c17f480"], custom("f_odd", 3, 5, 17, heads=3),
+                    custom("f_t1", 1, 9, 15), custom("f_t33", 33, 2, 3), custom("f_t64", 64, 1, 5),
+                    custom("f_hw1", 7, 1, 1), custom("f_b2", 4, 6, 7, batch=2)]
+
+LARGE = ["c81f480", "c81f720", "joint720"]
+
+
+# ------------------------------------------------------------------ RoPE
+
+@pytest.mark.parametrize("w", [si.WORKLOADS["tiny"], si.WORKLOADS["c17f480"],
+                               custom("r_joint", 2, 6, 10, n_text=37, dims=(16, 56, 56))],
+                         ids=lambda w: w.name)
+def test_rope3d_apply_matches_oracle(va, w):
+    q, _, _ = si.qkv(w)
+    x = dev(q)
+    y = va.rope3d_apply(x, vgrid(va, w))
+    ref = oracle.rope3d(q, ogrid(w))
+    got = host(y)
+    # one bf16 rounding of an fp32 result: within one bf16 ulp of the fp64 value
+    bound = 2.0 ** -7 * np.abs(ref) + 1e-6
+    assert (np.abs(got - ref) <= bound).all()
+    # in place gives the same bits
+    va.rope3d_apply(x, vgrid(va, w), out=x)
+    assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+
+
+# ------------------------------------------------------------- full / joint
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_full_attention_all_rows(va, w):
+    q, k, v = si.qkv(w)
+    o, lse = va.attn3d_full_fwd(dev(q), dev(k), dev(v), vgrid(va, w), return_lse=True)
+    ref, ref_lse = oracle.attention(q, k, v, ogrid(w), want_lse=True)
+    check(host(o).reshape(ref.shape), ref, f"full {w.name}")
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(ref_lse.shape), ref_lse, atol=2e-3, rtol=0)
+    assert va.device_error() == 0
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_full_attention_sampled_rows_full_size(va, name):
+    w = si.WORKLOADS[name]
+    q, k, v = si.qkv(w)
+    rows = si.sample_rows(w, 512)
+    o = va.attn3d_full_fwd(dev(q), dev(k), dev(v), vgrid(va, w))
+    got = host(o[:, :, torch.from_numpy(rows).cuda(), :]).reshape(w.batch * w.heads, rows.size, 128)
+    ref = oracle.attention(q, k, v, ogrid(w), rows=rows)
+    check(got, ref, f"full {name}")
+    if w.n_text:
+        txt = rows >= w.n_video
+        check(got[:, txt], ref[:, txt], f"full {name} text rows")
+    assert va.device_error() == 0
+
+
+def test_prerotated_keys_give_identical_output(va):
+    w = si.WORKLOADS["c17f480"]
+    q, k, v = (dev(x) for x in si.qkv(w))
+    g = vgrid(va, w)
+    o1 = va.attn3d_full_fwd(q, k, v, g)
+    kr = va.rope3d_apply(k, g)
+    o2 = va.attn3d_full_fwd(q, kr, v, g, k_rotated=True)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+def test_scale_argument(va):
+    w = custom("scale", 2, 4, 6)
+    q, k, v = si.qkv(w)
+    o = va.attn3d_full_fwd(dev(q), dev(k), dev(v), vgrid(va, w), scale=0.3)
+    ref = oracle.attention(q, k, v, ogrid(w), scale=0.3)
+    check(host(o).reshape(ref.shape), ref, "scale 0.3")
+
+
+def test_repeat_calls_are_deterministic(va):
+    w = si.WORKLOADS["c17f480"]
+    q, k, v = (dev(x) for x in si.qkv(w))
+    g = vgrid(va, w)
+    a = va.attn3d_full_fwd(q, k, v, g)
+    b = va.attn3d_full_fwd(q, k, v, g)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# -------------------------------------------------------------- factorised
+
+@pytest.mark.parametrize("w", FACTORISED_SMALL, ids=lambda w: w.name)
+def test_factorised_all_rows(va, w):
+    q, k, v = si.qkv(w)
+    os_, ot = va.attn_factorized_fwd(dev(q), dev(k), dev(v), vgrid(va, w))
+    shape = (w.batch * w.heads, w.N, 128)
+    check(host(os_).reshape(shape), oracle.attention(q, k, v, ogrid(w), mode="spatial"),
+          f"spatial {w.name}")
+    check(host(ot).reshape(shape), oracle.attention(q, k, v, ogrid(w), mode="temporal"),
+          f"temporal {w.name}")
+    assert va.device_error() == 0
+
+
+def test_factorised_sampled_rows_full_size(va):
+    w = si.WORKLOADS["c81f720"]
+    q, k, v = si.qkv(w)
+    rows = si.sample_rows(w, 512)
+    os_, ot = va.attn_factorized_fwd(dev(q), dev(k), dev(v), vgrid(va, w))
+    idx = torch.from_numpy(rows).cuda()
+    for mode, out in (("spatial", os_), ("temporal", ot)):
+        got = host(out[:, :, idx, :]).reshape(w.heads, rows.size, 128)
+        ref = oracle.attention(q, k, v, ogrid(w), mode=mode, rows=rows)
+        check(got, ref, f"{mode} c81f720")
+
+
+def test_factorised_single_pass_outputs(va):
+    w = si.WORKLOADS["tiny"]
+    q, k, v = (dev(x) for x in si.qkv(w))
+    g = vgrid(va, w)
+    s_only, none = va.attn_factorized_fwd(q, k, v, g, temporal=False)
+    assert none is None
+    none, t_only = va.attn_factorized_fwd(q, k, v, g, spatial=False)
+    s2, t2 = va.attn_factorized_fwd(q, k, v, g)
+    assert torch.equal(s_only.view(torch.int16), s2.view(torch.int16))
+    assert torch.equal(t_only.view(torch.int16), t2.view(torch.int16))
+
+
+def test_binding_rejects_bad_tensors(va):
+    g = va.Grid.make(2, 4, 4)
+    x = torch.zeros(1, 2, 32, 128, dtype=torch.float16, device="cuda")
+    with pytest.raises(TypeError):
+        va.attn3d_full_fwd(x, x, x, g)
+    y = torch.zeros(1, 2, 33, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(va.VA3DError):
+        va.attn3d_full_fwd(y, y, y, g)    # N inconsistent with the grid

@@ -1,0 +1,145 @@
+"""Host-side checks of the C-ABI library: it builds, loads without a GPU,
+exports every entry point the header declares, rejects bad arguments before
+touching a device, and has no CPU fallback."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "va3d.h")
+PKG = os.path.join(ROOT, "full_spatiotemporal_attention_b200")
+
+
+@pytest.fixture(scope="module")
+def va():
+    from full_spatiotemporal_attention_b200 import build
+    build.build()
+    import full_spatiotemporal_attention_b200 as va
+    return va
+
+
+def header_functions():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:const\s+char\s*\*|int|size_t)\s*(\w+)\s*\(", txt, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = header_functions()
+    for must in ("rope3d_apply", "attn3d_full_fwd", "attn_factorized_fwd",
+                 "va3d_grid_from_video", "va3d_workspace_bytes", "va3d_status_string",
+                 "va3d_device_error", "va3d_version"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(va):
+    out = subprocess.run(["nm", "-D", "--defined-only", va.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for name in header_functions():
+        assert name in exported, name
+        getattr(va.lib, name)           # resolvable through ctypes too
+    assert set(va.SYMBOLS) == set(header_functions())
+
+
+def test_library_needs_no_driver_to_load(va):
+    out = subprocess.run(["ldd", va.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out      # driver entry points are resolved at run time
+
+
+def test_grid_from_video_matches_oracle(va):
+    import oracle
+    for frames, h, w in [(81, 480, 832), (81, 720, 1280), (129, 720, 1280), (17, 480, 832),
+                         (1, 16, 16), (5, 64, 32)]:
+        g = va.grid_from_video(frames, h, w)
+        assert (g.T, g.H, g.W) == oracle.patch_grid(frames, h, w)
+        assert (g.d_t, g.d_h, g.d_w, g.theta) == (44, 42, 42, 10000.0)
+    g = va.grid_from_video(129, 720, 1280, dims=(16, 56, 56), n_text=256)
+    assert g.N == 118800 + 256
+
+
+@pytest.mark.parametrize("frames,h,w", [(80, 480, 832), (81, 1080, 1920), (81, 480, 840),
+                                        (0, 480, 832), (81, 8, 832)])
+def test_grid_from_video_rejects_off_grid_clips(va, frames, h, w):
+    with pytest.raises(va.VA3DError):
+        va.grid_from_video(frames, h, w)
+
+
+def test_workspace_bytes(va):
+    g = va.Grid.make(21, 30, 52)
+    tab = 8 * (21 * 22 + 30 * 21 + 52 * 21)
+    tab = (tab + 255) // 256 * 256
+    assert va.workspace_bytes(1, 12, 32760, g) == tab + 12 * 32760 * 256
+    assert va.workspace_bytes(1, 12, 32760, g, k_rotated=True) == tab
+    assert va.workspace_bytes(1, 12, 32761, g) == 0          # N inconsistent with the grid
+    bad = va.Grid.make(21, 30, 52, dims=(44, 42, 40))
+    assert va.workspace_bytes(1, 12, 32760, bad) == 0
+
+
+def test_status_strings(va):
+    for code in range(0, -7, -1):
+        assert va.lib.va3d_status_string(code)
+    assert va.lib.va3d_version() >= 100
+
+
+def test_bad_arguments_rejected_before_any_device_call(va):
+    lib = va.lib
+    g = va.Grid.make(2, 4, 4)
+    buf = ctypes.create_string_buffer(4096 + 16)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 15) // 16 * 16)
+    gp = ctypes.byref(g)
+    # head_dim other than 128
+    assert lib.attn3d_full_fwd(p, p, p, p, None, 1, 2, 32, 64, gp, 0.0, 0, p, 4096, None) == -2
+    # null input
+    assert lib.attn3d_full_fwd(None, p, p, p, None, 1, 2, 32, 128, gp, 0.0, 0, p, 4096, None) == -1
+    # N inconsistent with the grid
+    assert lib.attn3d_full_fwd(p, p, p, p, None, 1, 2, 33, 128, gp, 0.0, 0, p, 4096, None) == -1
+    # misaligned output
+    q = ctypes.c_void_p(p.value + 2)
+    assert lib.attn3d_full_fwd(p, p, p, q, None, 1, 2, 32, 128, gp, 0.0, 0, p, 4096, None) == -3
+    # workspace too small
+    assert lib.attn3d_full_fwd(p, p, p, p, None, 1, 2, 32, 128, gp, 0.0, 0, p, 16, None) == -4
+    # unknown flag
+    assert lib.attn3d_full_fwd(p, p, p, p, None, 1, 2, 32, 128, gp, 0.0, 8, p, 1 << 20, None) == -1
+    # factorised passes take no text tokens; temporal needs T' <= 64
+    gt = va.Grid.make(2, 4, 4, n_text=3)
+    assert lib.attn_factorized_fwd(p, p, p, p, p, 1, 2, 35, 128, ctypes.byref(gt), 0.0, 0, p,
+                                   1 << 20, None) == -1
+    gl = va.Grid.make(65, 1, 1)
+    assert lib.attn_factorized_fwd(p, p, p, None, p, 1, 1, 65, 128, ctypes.byref(gl), 0.0, 0, p,
+                                   1 << 20, None) == -2
+    # odd RoPE range
+    godd = va.Grid.make(2, 4, 4, dims=(43, 43, 42))
+    assert lib.rope3d_apply(p, p, 1, 2, 32, 128, ctypes.byref(godd), None) == -1
+
+
+def test_binding_has_no_cpu_path(va):
+    import torch
+    g = va.Grid.make(2, 4, 4)
+    x = torch.zeros(1, 2, 32, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        va.attn3d_full_fwd(x, x, x, g)
+    with pytest.raises(ValueError, match="CUDA"):
+        va.rope3d_apply(x, g)
+    with pytest.raises(ValueError, match="CUDA"):
+        va.attn_factorized_fwd(x, x, x, g)
+
+
+def test_product_and_oracle_share_nothing():
+    """The CUDA path never refers to the oracle or the input generator, and
+    the oracle never refers to the product."""
+    for dirpath, _, files in os.walk(PKG):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in txt.lower(), f
+                assert "seeded_inputs" not in txt, f
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        if f.endswith((".py", ".c")):
+            txt = open(os.path.join(ROOT, "oracle", f)).read()
+            assert "full_spatiotemporal_attention_b200" not in txt
+            assert "va3d.h" not in txt and "libva3d" not in txt
