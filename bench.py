@@ -37,8 +37,8 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="c81f480")
     p.add_argument("--e2e-steps", type=int, default=10)
@@ -90,7 +90,7 @@ def recorded_traffic(kernel, workload):
 
 class ClockSampler:
     """Samples nvidia-smi clocks and throttle reasons during the timed region."""
-    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    FIELDS = ("timestamp,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
@@ -102,11 +102,12 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (FileNotFoundError, OSError):
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
+        """Stop sampling; keep the samples taken between wall times t0 and t1."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -119,14 +120,19 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.splitlines():
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 8 or (self.uuid and parts[0] != self.uuid):
+            if len(parts) < 9 or (self.uuid and parts[1] != self.uuid):
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                clk, cmax = float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for name, val in zip(names, parts[4:8]):
+            if t0 is not None and not (t0 - 0.05 <= ts <= t1 + 0.05):
+                continue
+            sm.append(clk)
+            mx = cmax
+            for name, val in zip(names, parts[5:9]):
                 if val.lower() == "active":
                     reasons.add(name)
         if not sm:
@@ -192,9 +198,11 @@ def cpu_baseline(w, q, k, v, rows_per_head):
             "extrapolated_full_forward_s": round(dt * w.N / rows.size, 1)}
 
 
-def timed_loop(fn, steps, warmup, world, device, marks=False):
+def timed_loop(fn, steps, warmup, world, device, window=None):
     """Run fn(i) warmup times untimed, then `steps` times between CUDA events.
-    fn may return a pair of events bracketing its dominant kernel."""
+    fn may return a pair of events bracketing its dominant kernel.  If
+    `window` is a list, the wall-clock start and end of the timed region are
+    appended to it."""
     import torch
     for i in range(warmup):
         fn(i)
@@ -203,6 +211,8 @@ def timed_loop(fn, steps, warmup, world, device, marks=False):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     inner = []
+    if window is not None:
+        window.append(time.time())
     start.record()
     for i in range(steps):
         ev = fn(i)
@@ -210,6 +220,8 @@ def timed_loop(fn, steps, warmup, world, device, marks=False):
             inner.append(ev)
     end.record()
     torch.cuda.synchronize()
+    if window is not None:
+        window.append(time.time())
     barrier(world)
     total = start.elapsed_time(end)
     inner_ms = [a.elapsed_time(b) for a, b in inner]
@@ -250,9 +262,10 @@ def bench_ours(args, rank, world, local):
         pass
     sampler = ClockSampler(uuid)
     sampler.start()
-    time.sleep(0.3)
-    step_ms, attn_ms = timed_loop(step, args.steps, args.warmup, world, device)
-    clocks = sampler.stop()
+    time.sleep(0.5)
+    window = []
+    step_ms, attn_ms = timed_loop(step, args.steps, args.warmup, world, device, window=window)
+    clocks = sampler.stop(*window)
     step_ms = max_over_ranks(step_ms, world, device)
     attn_ms = max_over_ranks(attn_ms, world, device)
 

@@ -88,9 +88,13 @@ def test_rope3d_apply_matches_oracle(va, w):
     y = va.rope3d_apply(x, vgrid(va, w))
     ref = oracle.rope3d(q, ogrid(w))
     got = host(y)
-    # one bf16 rounding of an fp32 result: within one bf16 ulp of the fp64 value
-    bound = 2.0 ** -7 * np.abs(ref) + 1e-6
-    assert (np.abs(got - ref) <= bound).all()
+    # One bf16 rounding of an fp32 result (one bf16 ulp), plus the fp32 angle
+    # error: pos * inv_freq is rounded twice in fp32 (<= ~1e-5 rad for
+    # positions below 100), which moves a pair by that angle times its norm.
+    pair = np.sqrt(ref[..., 0::2] ** 2 + ref[..., 1::2] ** 2).repeat(2, axis=-1)
+    bound = 2.0 ** -7 * np.abs(ref) + 2e-5 * pair + 1e-7
+    err = np.abs(got - ref)
+    assert (err <= bound).all(), float((err - bound).max())
     # in place gives the same bits
     va.rope3d_apply(x, vgrid(va, w), out=x)
     assert torch.equal(x.view(torch.int16), y.view(torch.int16))
@@ -134,11 +138,18 @@ def test_prerotated_keys_give_identical_output(va):
 
 
 def test_scale_argument(va):
+    """A caller-given scale.  Rounding the rotated Q and K to bf16 perturbs each
+    logit in proportion to the scale, so the absolute bounds grow by
+    scale / (1/sqrt(128)) (3.4x at 0.3); the relative L2 bound stays."""
     w = custom("scale", 2, 4, 6)
     q, k, v = si.qkv(w)
     o = va.attn3d_full_fwd(dev(q), dev(k), dev(v), vgrid(va, w), scale=0.3)
     ref = oracle.attention(q, k, v, ogrid(w), scale=0.3)
-    check(host(o).reshape(ref.shape), ref, "scale 0.3")
+    got = host(o).reshape(ref.shape)
+    amp = 0.3 * np.sqrt(128.0)
+    err = np.abs(got - ref)
+    assert err.max() <= MAX_ABS * amp and err.mean() <= MEAN_ABS * amp
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= REL_L2
 
 
 def test_repeat_calls_are_deterministic(va):
