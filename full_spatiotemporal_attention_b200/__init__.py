@@ -28,7 +28,7 @@ HEAD_DIM = 128
 
 SYMBOLS = ("va3d_status_string", "va3d_version", "va3d_grid_from_video",
            "va3d_workspace_bytes", "rope3d_apply", "attn3d_full_fwd",
-           "attn_factorized_fwd", "va3d_device_error")
+           "attn_factorized_fwd", "va3d_device_error", "attn3d_full_fwd_noalloc")
 
 
 class VA3DError(RuntimeError):
@@ -79,6 +79,7 @@ def _load():
     lib.attn3d_full_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp, sz, vp]
     lib.attn_factorized_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp, sz, vp]
     lib.va3d_device_error.argtypes = [i]
+    lib.attn3d_full_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp]
     return lib
 
 
@@ -188,6 +189,29 @@ def attn3d_full_fwd(q, k, v, grid, *, scale=None, return_lse=False, k_rotated=Fa
                              ws.numel() * ws.element_size(), _stream(q))
     if rc != VA3D_OK:
         raise VA3DError("attn3d_full_fwd", rc)
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
+def attn3d_full_fwd_noalloc(q, k, v, grid, *, scale=None, return_lse=False, k_rotated=False,
+                            out=None, lse=None):
+    """attn3d_full_fwd using the library's built-in 64 MiB scratch instead of a
+    workspace (for callers that cannot allocate device memory); calls that
+    overlap in time on the GPU race on that scratch."""
+    torch = _torch()
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    B, H, N, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = lib.attn3d_full_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
+                                     ctypes.byref(grid), float(scale or 0.0),
+                                     VA3D_K_ROTATED if k_rotated else 0, _stream(q))
+    if rc != VA3D_OK:
+        raise VA3DError("attn3d_full_fwd_noalloc", rc)
     return (out, lse) if (return_lse or lse is not None) else out
 
 

@@ -259,6 +259,8 @@ const char *va3d_status_string(int status) {
     case VA3D_ERR_WORKSPACE: return "workspace missing or too small";
     case VA3D_ERR_CUDA: return "CUDA runtime or driver call failed";
     case VA3D_ERR_DEVICE: return "current device is not compute capability 10.0 (B200)";
+    case VA3D_ERR_SCRATCH_LIMIT:
+        return "problem needs more scratch than the 64 MiB built into attn3d_full_fwd_noalloc";
     default: return "unknown status";
     }
 }
@@ -356,3 +358,53 @@ int va3d_device_error(int reset) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Entry point without a caller workspace, for callers that cannot allocate
+// device memory.  Its scratch is this one static device array; every GPU that
+// loads the library holds it until the process exits.  In host code the
+// array's name is only a host-side stand-in, so the device address is looked
+// up with cudaGetSymbolAddress, once per device with that device current, and
+// cached.  Nothing in the scratch needs to start at zero: the table and the
+// rotated keys are written before they are read on every call.
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[VA3D_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[kMaxDevices] = {};
+
+int noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return VA3D_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return VA3D_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+            return VA3D_ERR_CUDA;
+        g_noalloc_addr[dev] = ptr;
+    }
+    *out = g_noalloc_addr[dev];
+    return VA3D_OK;
+}
+
+}  // namespace
+
+extern "C" int attn3d_full_fwd_noalloc(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
+                                       va3d_bf16 *o, float *lse, int B, int heads, int N,
+                                       int head_dim, const va3d_grid_t *grid, float softmax_scale,
+                                       unsigned flags, void *stream) {
+    const size_t need = va3d_workspace_bytes(B, heads, N, head_dim, grid, flags);
+    if (need == 0)   // invalid sizes or grid: report them exactly as the workspace entry does
+        return attn3d_full_fwd(q, k, v, o, lse, B, heads, N, head_dim, grid, softmax_scale, flags,
+                               nullptr, 0, stream);
+    if (need > VA3D_NOALLOC_SCRATCH_BYTES) return VA3D_ERR_SCRATCH_LIMIT;
+    void *scratch = nullptr;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc != VA3D_OK) return rc;
+    return attn3d_full_fwd(q, k, v, o, lse, B, heads, N, head_dim, grid, softmax_scale, flags,
+                           scratch, VA3D_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -38,7 +38,8 @@
  *    faults surface at the caller's next synchronisation.  A device-side
  *    watchdog (every wait in the kernels is bounded) records a code that
  *    va3d_device_error() returns.
- *  - Entry points are thread-safe: they keep no mutable host state.
+ *  - Entry points are thread-safe.  They keep no mutable host state, except
+ *    attn3d_full_fwd_noalloc's per-device address cache (mutex-guarded).
  */
 #ifndef VA3D_H
 #define VA3D_H
@@ -68,7 +69,8 @@ enum {
     VA3D_ERR_ALIGNMENT = -3,    /* a pointer is not 16-byte aligned */
     VA3D_ERR_WORKSPACE = -4,    /* workspace missing or smaller than va3d_workspace_bytes */
     VA3D_ERR_CUDA = -5,         /* a CUDA runtime or driver call failed */
-    VA3D_ERR_DEVICE = -6        /* current device is not compute capability 10.0 */
+    VA3D_ERR_DEVICE = -6,       /* current device is not compute capability 10.0 */
+    VA3D_ERR_SCRATCH_LIMIT = -7 /* needs more than the built-in scratch of the no-alloc entry */
 };
 
 /* Flags for the attention entry points. */
@@ -165,6 +167,38 @@ int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 
                         va3d_bf16 *o_spatial, va3d_bf16 *o_temporal, int B, int heads, int N,
                         int head_dim, const va3d_grid_t *grid, float softmax_scale,
                         unsigned flags, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Capacity of the built-in scratch used by attn3d_full_fwd_noalloc. */
+#define VA3D_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * attn3d_full_fwd for callers that cannot allocate device memory and so cannot
+ * hand in a workspace: for example a plugin running inside a host framework
+ * that owns all device memory and passes in only its input and output
+ * pointers, or code on a path where calling cudaMalloc is not allowed or too
+ * slow.  (The pages have no counterpart; this is a property of the library.)
+ *
+ * Same arguments, results and errors as attn3d_full_fwd, minus the workspace.
+ * Its scratch (angle table and, unless VA3D_K_ROTATED, the rotated keys) lives
+ * in one static device array of VA3D_NOALLOC_SCRATCH_BYTES (64 MiB) built into
+ * the library; every GPU that loads the library holds that array until the
+ * process exits.  A call whose scratch need, va3d_workspace_bytes(B, heads,
+ * N, head_dim, grid, flags), exceeds 64 MiB returns VA3D_ERR_SCRATCH_LIMIT
+ * and launches nothing (without VA3D_K_ROTATED that is about
+ * B*heads*N <= 262,000 rows).  The function calls no allocator.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array, and each call overwrites the
+ * parts it reads before reading them, so leftovers of the previous call do no
+ * harm; but calls that overlap in time on the GPU (different streams, or
+ * different host threads, without ordering between them) race on the array
+ * and give wrong results.  Order them on one stream or synchronise.
+ */
+int attn3d_full_fwd_noalloc(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
+                            va3d_bf16 *o, float *lse, int B, int heads, int N, int head_dim,
+                            const va3d_grid_t *grid, float softmax_scale, unsigned flags,
+                            void *stream);
 
 /*
  * Last device-side watchdog code recorded on the current device
