@@ -58,19 +58,19 @@ def peaks():
         return FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(files):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "full_spatiotemporal_attention_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + fh.read())
+    for f in files:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (its `source_hash` line matches)."""
+    the current sources of that kernel (its `source_hash` over the listed
+    `source_files` matches); otherwise None."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_ncu.md")
     if not os.path.exists(path):
         return None
@@ -80,11 +80,11 @@ def recorded_traffic(kernel, workload):
             if ":" in line and line.startswith("- "):
                 key, _, val = line[2:].partition(":")
                 vals[key.strip()] = val.strip().strip("`")
-    if vals.get("source_hash") != kernel_source_hash():
-        return None
     try:
+        if vals.get("source_hash") != kernel_source_hash(vals["source_files"].split(",")):
+            return None
         return float(vals["dram_bytes_per_launch_full_size"])
-    except (KeyError, ValueError):
+    except (KeyError, ValueError, OSError):
         return None
 
 

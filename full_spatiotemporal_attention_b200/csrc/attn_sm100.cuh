@@ -14,12 +14,15 @@
 //   warps 4-7   softmax group 1: rows of query tile 1
 //   warp  8     tcgen05.mma issuer (one thread) and TMEM allocator
 //   warp  9     TMA loader (one thread)
+//   warps 10-11 idle (they complete the producer warpgroup for setmaxnreg)
 // TMEM (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1, 128 columns each;
 // P (bf16 pairs) overwrites the first 64 columns of its S.  The MMA issuer
 // ping-pongs the two query tiles so that one tile's softmax overlaps the
 // other tile's QK^T and PV products.  Q, K, V tiles are 128 rows x 128 bf16,
 // loaded by TMA as two 64-column boxes with the 128-byte swizzle.
 #pragma once
+
+#include <type_traits>
 
 #include "ptx.cuh"
 #include "rope.cuh"
@@ -31,7 +34,14 @@ constexpr int BM = 128;                    // query rows per tile
 constexpr int BN = 128;                    // keys per tile
 constexpr int HD = 128;                    // head dim
 constexpr int kStages = 2;                 // K and V ring depth
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;             // three warpgroups
+// Register split after launch (168 per thread at launch = 64,512 per block):
+// the two softmax warpgroups take 216, the producer warpgroup keeps 72;
+// 2 * 128 * 216 + 128 * 72 = 64,512.
+constexpr int kSoftmaxRegs = 216;
+constexpr int kProducerRegs = 72;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * 168,
+              "register split exceeds the launch allocation");
 constexpr int kTileBytes = BM * HD * 2;    // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2; // one 64-column box: 128 rows x 128 B
 
@@ -65,6 +75,9 @@ constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 384;
 // Lazy rescaling: a row keeps its running maximum (log2 units) until a new
 // score exceeds it by more than this; P values then stay below 2^8.
 constexpr float kRescaleThreshold = 8.0f;
+
+// Every kPolyEvery-th pair of scores takes the polynomial exp2 (FMA pipe).
+constexpr int kPolyEvery = 4;
 
 struct AttnArgs {
     int N;             // tokens per (batch, head) sequence
@@ -160,8 +173,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_TMEM_SLOT);
-
-    if (warp == 9) {
+    // Each role runs inside the branch that set its register budget (the new
+    // budget applies to the code that instruction dominates).
+    if (warp >= 8) {
+    regs_lower<kProducerRegs>();
+    if (warp >= 10) {
+        // idle
+    } else if (warp == 9) {
         // ------------------------------------------------------------ loader
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -172,8 +190,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 for (int hf = 0; hf < 2; ++hf)
                     tma_load_3d(sbase + OFF_Q + i * kTileBytes + hf * kHalfBytes, &tmQ,
                                 bar(B_QFULL), hf * 64, q0 + i * BM, bh);
-            int last_k[kStages] = {-1, -1};   // last key tile issued into each stage
-            int last_v[kStages] = {-1, -1};
+            // Tile j goes to stage j & 1 with phase (j >> 1) & 1; only the last
+            // kStages issued tiles can still be in flight or unreleased.
+            int k_issued = 0, v_issued = 0;
             bool ok = true;
             for (int j = 0; j < n_kv; ++j) {
                 const int s = j & 1;
@@ -186,7 +205,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 for (int hf = 0; hf < 2; ++hf)
                     tma_load_3d(sbase + OFF_K + s * kTileBytes + hf * kHalfBytes, &tmK,
                                 bar(B_KFULL0 + s), hf * 64, kv0, bh);
-                last_k[s] = j;
+                k_issued = j + 1;
                 if (j >= kStages &&
                     !(ok = mbar_wait(bar(B_VEMPTY0 + s), ph ^ 1, abort_flag, VA3D_DEVERR_TIMEOUT_LOAD)))
                     break;
@@ -194,27 +213,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 for (int hf = 0; hf < 2; ++hf)
                     tma_load_3d(sbase + OFF_V + s * kTileBytes + hf * kHalfBytes, &tmV,
                                 bar(B_VFULL0 + s), hf * 64, kv0, bh);
-                last_v[s] = j;
+                v_issued = j + 1;
             }
+            const int k_first = k_issued > kStages ? k_issued - kStages : 0;
+            const int v_first = v_issued > kStages ? v_issued - kStages : 0;
             if (ok) {
                 // Producer tail: wait until the last tile of each stage has been
                 // released, so no barrier arrival can land after the CTA exits.
-                for (int s = 0; s < kStages && ok; ++s) {
-                    if (last_k[s] >= 0)
-                        ok = mbar_wait(bar(B_KEMPTY0 + s), (last_k[s] >> 1) & 1, abort_flag,
-                                       VA3D_DEVERR_TIMEOUT_LOAD);
-                    if (ok && last_v[s] >= 0)
-                        ok = mbar_wait(bar(B_VEMPTY0 + s), (last_v[s] >> 1) & 1, abort_flag,
-                                       VA3D_DEVERR_TIMEOUT_LOAD);
-                }
+                for (int j = k_first; j < k_issued && ok; ++j)
+                    ok = mbar_wait(bar(B_KEMPTY0 + (j & 1)), (j >> 1) & 1, abort_flag,
+                                   VA3D_DEVERR_TIMEOUT_LOAD);
+                for (int j = v_first; j < v_issued && ok; ++j)
+                    ok = mbar_wait(bar(B_VEMPTY0 + (j & 1)), (j >> 1) & 1, abort_flag,
+                                   VA3D_DEVERR_TIMEOUT_LOAD);
             }
             if (!ok) {
                 // Let the copies already in flight land before the CTA exits.
                 mbar_wait_drain(bar(B_QFULL), 0);
-                for (int s = 0; s < kStages; ++s) {
-                    if (last_k[s] >= 0) mbar_wait_drain(bar(B_KFULL0 + s), (last_k[s] >> 1) & 1);
-                    if (last_v[s] >= 0) mbar_wait_drain(bar(B_VFULL0 + s), (last_v[s] >> 1) & 1);
-                }
+                for (int j = k_first; j < k_issued; ++j)
+                    mbar_wait_drain(bar(B_KFULL0 + (j & 1)), (j >> 1) & 1);
+                for (int j = v_first; j < v_issued; ++j)
+                    mbar_wait_drain(bar(B_VFULL0 + (j & 1)), (j >> 1) & 1);
             }
         }
     } else if (warp == 8) {
@@ -288,7 +307,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 mbar_wait_drain(bar(B_DRAIN), 0);
             }
         }
+    }
     } else {
+        regs_raise<kSoftmaxRegs>();
         // ---------------------------------------------------------- softmax
         const int g = warp >> 2;                  // query tile of this group
         const int r = ((warp & 3) << 5) + lane;   // row in the tile = TMEM lane
@@ -320,14 +341,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
             for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
             float *s = reinterpret_cast<float *>(sr);
-            if (j == n_kv - 1 && kv_last_valid < BN) {
+            const bool masked_tile = (j == n_kv - 1) && (kv_last_valid < BN);
+            if (masked_tile) {
 #pragma unroll
                 for (int c = 0; c < BN; ++c)
                     if (c >= kv_last_valid) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // row maximum: four independent chains of three-input max
+            float m4[4];
 #pragma unroll
-            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+            for (int q = 0; q < 4; ++q) {
+                const float *v = s + 32 * q;
+                float m = fmax3(v[0], v[1], v[2]);
+#pragma unroll
+                for (int c = 3; c < 31; c += 2) m = fmax3(m, v[c], v[c + 1]);
+                m4[q] = fmaxf(m, v[31]);
+            }
+            const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
             const float m_new = fmaxf(m_ref, mx * a.scale_log2);
             float alpha = 1.0f;
             const bool bump = m_new - m_ref > kRescaleThreshold;
@@ -335,20 +365,40 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 alpha = ex2(m_ref - m_new);
                 m_ref = m_new;
             }
-            const float neg_m = -m_ref;
-            float rowsum = 0.0f;
+            // P = 2^(s*scale - m) in pairs; a quarter of the pairs use the FMA-pipe
+            // exp2 to offload the MUFU unit (not on the masked tile, whose -inf
+            // scores need an exact zero); four independent fp32x2 partial sums.
+            const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+            const float2 nm2 = make_float2(-m_ref, -m_ref);
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
+            auto exp_store = [&](auto mixed) {
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t pk[32];
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2(fmaf(s[64 * hf + 2 * c], a.scale_log2, neg_m));
-                    const float p1 = ex2(fmaf(s[64 * hf + 2 * c + 1], a.scale_log2, neg_m));
-                    rowsum += p0 + p1;
-                    pk[c] = pack_bf16x2(p0, p1);
+                    for (int c = 0; c < 32; ++c) {
+                        const int e = 64 * hf + 2 * c;
+                        const float2 x = fma2(make_float2(s[e], s[e + 1]), sc2, nm2);
+                        float2 p;
+                        if (decltype(mixed)::value && (c % kPolyEvery) == kPolyEvery - 1)
+                            p = exp2_poly(x);
+                        else
+                            p = make_float2(ex2(x.x), ex2(x.y));
+                        acc[c & 3] = add2(acc[c & 3], p);
+                        pk[c] = pack_bf16x2(p.x, p.y);
+                    }
+                    tmem_st32(taS + 32 * hf, pk);
                 }
-                tmem_st32(taS + 32 * hf, pk);
-            }
+            };
+            if (masked_tile)
+                exp_store(std::false_type{});
+            else
+                exp_store(std::true_type{});
+            const float2 acc01 = add2(acc[0], acc[1]);
+            const float2 acc23 = add2(acc[2], acc[3]);
+            const float2 acc_all = add2(acc01, acc23);
+            const float rowsum = acc_all.x + acc_all.y;
             if (j > 0 && __any_sync(0xffffffffu, bump)) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {

@@ -121,6 +121,18 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
 
 // ------------------------------------------------------------------ tcgen05
 
+// Per-warpgroup register reallocation.  All warps of a warpgroup execute
+// it; the total over warpgroups must not exceed the block's launch allocation.
+template <int N>
+__device__ __forceinline__ void regs_raise() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <int N>
+__device__ __forceinline__ void regs_lower() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Allocate `ncols` TMEM columns (power of two >= 32); the base address is
 // written to shared memory at `slot`.  Executed by one full warp.
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
@@ -247,6 +259,67 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Packed fp32x2 arithmetic (sm_100): one instruction for two lanes of work.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// 2^x for a pair on the FMA pipe instead of the MUFU unit.  Range reduction
+// in the style of Cody and Waite: n = round(x) by adding 1.5 * 2^23 (the sum's
+// last mantissa bits then hold n), f = x - n in [-1/2, 1/2]; 2^f by a
+// degree-3 polynomial whose coefficients were fitted here for minimum
+// maximum relative error on [-1/2, 1/2] (7.5e-5, far below bf16's 2^-9
+// rounding of P); 2^n applied by adding n to the exponent field.  Inputs
+// must be <= 64; inputs below -120 are treated as -120 (2^-120 ~ 0 next to
+// the row sum, which is >= 1).
+__device__ __forceinline__ float2 exp2_poly(float2 x) {
+    x.x = fmaxf(x.x, -120.0f);
+    x.y = fmaxf(x.y, -120.0f);
+    const float2 shifter = make_float2(12582912.0f, 12582912.0f);
+    const float2 j = add2(x, shifter);
+    const float2 n = sub2(j, shifter);
+    const float2 f = sub2(x, n);
+    float2 p = fma2(f, make_float2(0.0551716685f, 0.0551716685f),
+                    make_float2(0.242611125f, 0.242611125f));
+    p = fma2(p, f, make_float2(0.693260968f, 0.693260968f));
+    p = fma2(p, f, make_float2(0.999928057f, 0.999928057f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

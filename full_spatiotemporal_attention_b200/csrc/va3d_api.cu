@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "va3d.h"
@@ -110,15 +111,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [BH, N, 128] bf16 viewed as a 3D tensor (dim, row, bh); boxes of
-// 64 columns x 128 rows with the 128-byte swizzle; rows past N read as zero.
-int make_map(CUtensorMap *map, const void *base, int N, int BH) {
+// 64 columns x box_rows rows with the 128-byte swizzle; rows past N read as zero.
+int make_map(CUtensorMap *map, const void *base, int N, int BH, int box_rows) {
     auto fn = encode_fn();
     if (fn == nullptr) return VA3D_ERR_CUDA;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(N),
                           static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2,
                              static_cast<cuuint64_t>(N) * kHeadDim * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -152,9 +153,9 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
                 cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     int rc;
-    if ((rc = make_map(&mq, q, N, BH)) != VA3D_OK) return rc;
-    if ((rc = make_map(&mk, k_rot, N, BH)) != VA3D_OK) return rc;
-    if ((rc = make_map(&mv, v, N, BH)) != VA3D_OK) return rc;
+    if ((rc = make_map(&mq, q, N, BH, fa::BM)) != VA3D_OK) return rc;
+    if ((rc = make_map(&mk, k_rot, N, BH, fa::BN)) != VA3D_OK) return rc;
+    if ((rc = make_map(&mv, v, N, BH, fa::BN)) != VA3D_OK) return rc;
     fa::AttnArgs a;
     std::memset(&a, 0, sizeof a);
     a.N = N;
@@ -178,23 +179,35 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
 
 template <int MAXT>
 int launch_temporal_t(const tp::TemporalArgs &a, cudaStream_t st) {
-    constexpr int smem = tp::Cfg<MAXT>::kSmemBytes;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return VA3D_ERR_CUDA;
+    // Warps per block and blocks per SM from the shared-memory budget; the
+    // grid is persistent (at most the resident blocks), each warp strides
+    // over (batch*head, position) tasks.
+    const int warp_bytes = tp::temporal_warp_bytes(a.T);
+    const int budget = tp::Cfg<MAXT>::kSmemBudget;
+    const int warps = std::max(1, std::min(tp::Cfg<MAXT>::kMaxWarps, budget / warp_bytes));
+    const int smem = warps * warp_bytes;
+    const int per_sm = std::max(1, std::min(4, (216 * 1024) / smem));
     if (cudaFuncSetAttribute(tp::temporal_kernel<MAXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return VA3D_ERR_CUDA;
     const long long tasks = static_cast<long long>(a.BH) * a.HW;
-    const long long blocks = (tasks + tp::Cfg<MAXT>::kWarps - 1) / tp::Cfg<MAXT>::kWarps;
-    if (blocks > 0x7fffffffll) return VA3D_ERR_UNSUPPORTED;
-    tp::temporal_kernel<MAXT><<<static_cast<unsigned>(blocks), tp::Cfg<MAXT>::kWarps * 32, smem, st>>>(a);
+    const long long need = (tasks + warps - 1) / warps;
+    const long long blocks = std::min<long long>(need, static_cast<long long>(sms) * per_sm);
+    tp::temporal_kernel<MAXT><<<static_cast<unsigned>(blocks), warps * 32, smem, st>>>(a);
     return launch_status();
 }
 
-int launch_temporal(const void *q, const void *k_rot, const void *v, void *o, int BH, int N,
-                    const RopeParams &rp, const float2 *tab, float scale, cudaStream_t st) {
+// k is the raw key tensor (rotated here) unless k_rotated.
+int launch_temporal(const void *q, const void *k, bool k_rotated, const void *v, void *o, int BH,
+                    int N, const RopeParams &rp, const float2 *tab, float scale, cudaStream_t st) {
     tp::TemporalArgs a;
     std::memset(&a, 0, sizeof a);
     a.q = static_cast<const __nv_bfloat16 *>(q);
-    a.k = static_cast<const __nv_bfloat16 *>(k_rot);
+    a.k = static_cast<const __nv_bfloat16 *>(k);
     a.v = static_cast<const __nv_bfloat16 *>(v);
     a.o = static_cast<__nv_bfloat16 *>(o);
     a.N = N;
@@ -202,7 +215,7 @@ int launch_temporal(const void *q, const void *k_rot, const void *v, void *o, in
     a.HW = rp.HW;
     a.BH = BH;
     a.scale_log2 = static_cast<float>(scale * kLog2e);
-    a.rope_q = 1;
+    a.rope_k = k_rotated ? 0 : 1;
     a.rope_tab = tab;
     a.rp = rp;
     if (rp.T <= 32) return launch_temporal_t<32>(a, st);
@@ -220,7 +233,7 @@ struct Prepared {
 
 int prepare(const void *q, const void *k, const void *v, int B, int heads, int N, int head_dim,
             const va3d_grid_t *grid, float softmax_scale, unsigned flags, void *workspace,
-            size_t workspace_bytes, cudaStream_t st, Prepared *out) {
+            size_t workspace_bytes, bool need_k_rot, cudaStream_t st, Prepared *out) {
     int rc;
     if ((rc = check_sizes(B, heads, N, head_dim)) != VA3D_OK) return rc;
     if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
@@ -238,6 +251,8 @@ int prepare(const void *q, const void *k, const void *v, int B, int heads, int N
     if ((rc = launch_table(static_cast<float2 *>(workspace), out->rp, st)) != VA3D_OK) return rc;
     if (flags & VA3D_K_ROTATED) {
         out->k_rot = k;
+    } else if (!need_k_rot) {
+        out->k_rot = nullptr;
     } else {
         void *kr = static_cast<uint8_t *>(workspace) + table_bytes(grid);
         if ((rc = launch_rope(k, kr, B * heads, N, out->rp, st)) != VA3D_OK) return rc;
@@ -314,7 +329,7 @@ int attn3d_full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Prepared p;
     int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
-                     workspace_bytes, st, &p);
+                     workspace_bytes, true, st, &p);
     if (rc != VA3D_OK) return rc;
     return launch_attn(q, p.k_rot, v, o, lse, B * heads, N, N, 1, p.rp, p.tab, p.scale, st);
 }
@@ -332,7 +347,7 @@ int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Prepared p;
     int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
-                     workspace_bytes, st, &p);
+                     workspace_bytes, o_spatial != nullptr, st, &p);
     if (rc != VA3D_OK) return rc;
     if (o_spatial != nullptr) {
         rc = launch_attn(q, p.k_rot, v, o_spatial, nullptr, B * heads, N, p.rp.HW, p.rp.T, p.rp,
@@ -340,7 +355,8 @@ int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 
         if (rc != VA3D_OK) return rc;
     }
     if (o_temporal != nullptr)
-        rc = launch_temporal(q, p.k_rot, v, o_temporal, B * heads, N, p.rp, p.tab, p.scale, st);
+        rc = launch_temporal(q, k, (flags & VA3D_K_ROTATED) != 0, v, o_temporal, B * heads, N, p.rp,
+                             p.tab, p.scale, st);
     return rc;
 }
 
