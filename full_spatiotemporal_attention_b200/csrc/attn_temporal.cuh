@@ -5,7 +5,7 @@
 //
 // The pass is HBM-bound (each position reads T' rows of Q, K, V and writes T'
 // rows of O; its 4*T'^2*d FLOPs are small), so the design goal is streaming:
-//  - persistent warps (up to 16 per SM, as many as shared memory holds), one
+//  - persistent warps (up to 12 per block, as many as shared memory holds), one
 //    (batch*head, position) task at a time, rows fetched with 16-byte
 //    cp.async (each row is 256 contiguous bytes); the other resident warps
 //    compute while one waits for its rows;
@@ -102,40 +102,110 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Largest |x| over bf16 bit patterns, as a bit pattern (sign cleared); the
-// ordering of such patterns follows the ordering of magnitudes.
-__device__ __forceinline__ uint32_t absmax_bits(uint4 v, uint32_t m) {
-    const uint32_t k = 0x7FFF7FFFu;
-    uint32_t a = __vmaxu2(__vmaxu2(v.x & k, v.y & k), __vmaxu2(v.z & k, v.w & k));
-    return max(m, max(a & 0xFFFFu, a >> 16));
-}
-
-// Power-of-two exponent s such that every rotated element, scaled by 2^s, is
-// below 2^14: |x| < 2^(e-126) for a bf16 exponent field e, a rotation can
-// grow one element by at most sqrt(2).  Clamped so the combined scale of two
-// operands stays a normal float.
-__device__ __forceinline__ int fp16_scale_exponent(uint32_t absmax_bits) {
-    const int e = static_cast<int>((absmax_bits >> 7) & 0xFF);
-    return max(-60, min(60, 139 - e));
-}
-
 __device__ __forceinline__ float pow2f(int s) {
     return __uint_as_float(static_cast<uint32_t>(127 + s) << 23);
 }
 
 template <int MAXT>
 struct Cfg {
-    static constexpr int kMaxWarps = 16;
+    // Up to 12 warps (168 registers each); at T' = 64 shared memory holds 4.
+    static constexpr int kMaxWarps = 12;
     static constexpr int kSmemBudget = 208 * 1024;
 };
 
 // Shared memory per warp: (Q, K, V) with T rows of 256 bytes.
 __host__ __device__ inline int temporal_warp_bytes(int T) { return 3 * T * 256; }
 
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// One rotated pair (x0 c - x1 s, x0 s + x1 c) times a power-of-two scale,
+// where cs holds (c * scale, s * scale); returned as packed fp16.  m tracks
+// the largest magnitude of the unscaled rotated values (cs / scale).
+__device__ __forceinline__ uint32_t rot_f16(uint32_t packed_bf16, float2 cs) {
+    const float2 x = unpack_bf16x2(packed_bf16);
+    const float2 y = fma2(x, make_float2(cs.x, cs.x), mul2(make_float2(-x.y, x.x), make_float2(cs.y, cs.y)));
+    return pack_f16x2(y.x, y.y);
+}
+
+__device__ __forceinline__ uint32_t rot_f16_max(uint32_t packed_bf16, float2 cs, float &m) {
+    const float2 x = unpack_bf16x2(packed_bf16);
+    const float2 y = fma2(x, make_float2(cs.x, cs.x), mul2(make_float2(-x.y, x.x), make_float2(cs.y, cs.y)));
+    m = fmax3(m, fabsf(y.x), fabsf(y.y));
+    return pack_f16x2(y.x, y.y);
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// fp16 is used as is when the largest rotated magnitude lies in
+// [2^-6, 2^15); outside that range the operand is redone with a power of two
+// that brings its largest magnitude into [2^13, 2^14).
+__device__ __forceinline__ bool fp16_range_ok(float m) {
+    return m == 0.0f || (m >= 0.015625f && m < 32768.0f);
+}
+
+__device__ __forceinline__ int fp16_rescale_exponent(float m) {
+    const int e = static_cast<int>((__float_as_uint(m) >> 23) & 0xFF) - 127;   // m in [2^e, 2^(e+1))
+    return max(-60, min(60, 13 - e));
+}
+
+// RoPE + fp16 in place for the T rows of one staged operand (raw bf16 rows
+// in shared memory).  Scale 1 unless the largest rotated magnitude is out of
+// fp16's comfortable range; then the rows are read again from global memory
+// and redone with a power-of-two scale, whose exponent is returned.
+template <bool kRotate>
+__device__ __forceinline__ int rotate_to_f16(uint8_t *tile, const __nv_bfloat16 *src, size_t base,
+                                             size_t tstride, int T, int rlane, int cch,
+                                             const float2 (&cs_fixed)[4], const bool (&is_t)[4],
+                                             const TemporalArgs &a, bool rotate) {
+    auto angle = [&](int r, int e) -> float2 {
+        if (!rotate) return make_float2(1.f, 0.f);
+        return is_t[e] ? a.rope_tab[r * a.rp.half_t + cch * 4 + e] : cs_fixed[e];
+    };
+    float mx = 0.f;
+    for (int r = rlane; r < T; r += 2) {
+        uint4 *p = reinterpret_cast<uint4 *>(tile + swz(r, cch));
+        const uint4 x = *p;
+        *p = make_uint4(rot_f16_max(x.x, angle(r, 0), mx), rot_f16_max(x.y, angle(r, 1), mx),
+                        rot_f16_max(x.z, angle(r, 2), mx), rot_f16_max(x.w, angle(r, 3), mx));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (fp16_range_ok(mx)) return 0;
+    const int ex = fp16_rescale_exponent(mx);
+    const float sc = pow2f(ex);
+    for (int r = rlane; r < T; r += 2) {
+        const uint4 x = ldg_stream(src + base + r * tstride + cch * 8);
+        float2 c[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            c[e] = angle(r, e);
+            c[e] = make_float2(c[e].x * sc, c[e].y * sc);
+        }
+        *reinterpret_cast<uint4 *>(tile + swz(r, cch)) =
+            make_uint4(rot_f16(x.x, c[0]), rot_f16(x.y, c[1]), rot_f16(x.z, c[2]), rot_f16(x.w, c[3]));
+    }
+    return ex;
+}
+
 template <int MAXT>
 __global__ void __launch_bounds__(Cfg<MAXT>::kMaxWarps * 32)
 temporal_kernel(const __grid_constant__ TemporalArgs a) {
-    constexpr int NP = MAXT / 16;   // pairs of n8 key tiles (and k16 steps over keys)
+    constexpr int NP = MAXT / 16;   // pairs of n8 key tiles and k16 key steps
+    constexpr int MG = 2;           // query m-tiles computed together
     extern __shared__ __align__(16) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -146,64 +216,36 @@ temporal_kernel(const __grid_constant__ TemporalArgs a) {
     long long task = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + warp;
     if (task >= total) return;   // the whole warp leaves together; no block barrier is used
 
-    uint8_t *wbase = smem + warp * temporal_warp_bytes(T);
+    uint8_t *sq = smem + warp * temporal_warp_bytes(T);   // Q (raw, fp16 rotated, then bf16 O)
+    uint8_t *sk = sq + tensor_bytes;                     // K (raw, then fp16 rotated)
+    uint8_t *sv = sk + tensor_bytes;                     // V (bf16)
+    const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv);
     const size_t tstride = static_cast<size_t>(a.HW) * 128;   // elements between frames
 
-    auto row0 = [&](long long tk) -> size_t {   // element offset of frame 0 of a task
-        const long long bh = tk / a.HW;
-        const long long pos = tk - bh * a.HW;
-        return (static_cast<size_t>(bh) * a.N + static_cast<size_t>(pos)) * 128;
-    };
-    auto issue = [&](long long tk, int) {
-        const size_t base = row0(tk);
-        const uint32_t s0 = smem_u32(wbase);
-        for (int idx = lane; idx < T * 16; idx += 32) {
-            const int r = idx >> 4, c = idx & 15;
-            const uint32_t off = swz(r, c);
-            const size_t g = base + r * tstride + c * 8;
-            cp_async16(s0 + off, a.q + g);
-            cp_async16(s0 + tensor_bytes + off, a.k + g);
-            cp_async16(s0 + 2 * tensor_bytes + off, a.v + g);
-        }
-        cp_async_commit();
-    };
-
-    const int g = lane >> 2;   // fragment row
-    const int tq = lane & 3;   // fragment column pair
-    // In the RoPE and scale passes a lane always handles the same 16-byte
-    // chunk (pairs 4c .. 4c+3) of rows (lane >> 4), (lane >> 4) + 2, ...
+    const int g = lane >> 2;      // mma fragment row
+    const int tq = lane & 3;      // mma fragment column pair
+    // In the copy and rotate passes lane handles 16-byte chunk cch (pairs
+    // 4cch..4cch+3) of rows rlane, rlane + 2, ...
     const int cch = lane & 15;
     const int rlane = lane >> 4;
-    uint8_t *sq = wbase;
-    uint8_t *sk = sq + tensor_bytes;
-    uint8_t *sv = sk + tensor_bytes;
-    const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv);
+    const int tl = T - 1;
+    const int n_mt = (T + 15) >> 4;
+
     for (; task < total; task += stride) {
-        issue(task, 0);
-        cp_async_wait<0>();
-        __syncwarp();
         const long long bh = task / a.HW;
         const int pos = static_cast<int>(task - bh * a.HW);
+        const size_t base = (static_cast<size_t>(bh) * a.N + static_cast<size_t>(pos)) * 128;
 
-        // ---- per-task fp16 scales for Q and K
-        uint32_t mq = 0, mk = 0;
-#pragma unroll 4
         for (int r = rlane; r < T; r += 2) {
+            const size_t gofs = base + r * tstride + cch * 8;
             const uint32_t off = swz(r, cch);
-            mq = absmax_bits(*reinterpret_cast<const uint4 *>(sq + off), mq);
-            mk = absmax_bits(*reinterpret_cast<const uint4 *>(sk + off), mk);
+            cp_async16(aq + off, a.q + gofs);
+            cp_async16(ak + off, a.k + gofs);
+            cp_async16(av + off, a.v + gofs);
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            mq = max(mq, __shfl_xor_sync(0xffffffffu, mq, o));
-            mk = max(mk, __shfl_xor_sync(0xffffffffu, mk, o));
-        }
-        const int eq = fp16_scale_exponent(mq), ek = fp16_scale_exponent(mk);
-        const float sq_f = pow2f(eq), sk_f = pow2f(ek);
-        const float scale_log2 = a.scale_log2 * pow2f(-(eq + ek));
+        cp_async_commit();
 
-        // ---- rotate (RoPE) and convert Q and K to scaled fp16 in place.
-        // Angles of h and w pairs are fixed for the task; t pairs vary by row.
+        // angles: h and w pairs are fixed for the task, t pairs vary per row
         const int h = pos / a.rp.W;
         const int w = pos - h * a.rp.W;
         float2 cs_fixed[4];
@@ -214,134 +256,136 @@ temporal_kernel(const __grid_constant__ TemporalArgs a) {
             is_t[e] = p < a.rp.pe_t;
             cs_fixed[e] = is_t[e] ? make_float2(1.f, 0.f) : a.rope_tab[table_index(a.rp, p, 0, h, w)];
         }
-#pragma unroll 2
-        for (int r = rlane; r < T; r += 2) {
-            const uint32_t off = swz(r, cch);
-            uint4 *pq = reinterpret_cast<uint4 *>(sq + off);
-            uint4 *pk = reinterpret_cast<uint4 *>(sk + off);
-            uint4 vq = *pq, vk = *pk;
-            uint32_t *eqv = reinterpret_cast<uint32_t *>(&vq);
-            uint32_t *ekv = reinterpret_cast<uint32_t *>(&vk);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 cs = is_t[e] ? a.rope_tab[r * a.rp.half_t + cch * 4 + e] : cs_fixed[e];
-                const float2 x = unpack_bf16x2(eqv[e]);
-                eqv[e] = pack_f16x2((x.x * cs.x - x.y * cs.y) * sq_f, (x.x * cs.y + x.y * cs.x) * sq_f);
-                const float2 y = unpack_bf16x2(ekv[e]);
-                if (a.rope_k)
-                    ekv[e] = pack_f16x2((y.x * cs.x - y.y * cs.y) * sk_f, (y.x * cs.y + y.y * cs.x) * sk_f);
-                else
-                    ekv[e] = pack_f16x2(y.x * sk_f, y.y * sk_f);
-            }
-            *pq = vq;
-            *pk = vk;
-        }
+        cp_async_wait<0>();
+        __syncwarp();
+        const int eq = rotate_to_f16<true>(sq, a.q, base, tstride, T, rlane, cch, cs_fixed, is_t, a, true);
+        const int ek = rotate_to_f16<true>(sk, a.k, base, tstride, T, rlane, cch, cs_fixed, is_t, a,
+                                           a.rope_k != 0);
+        const float scale_log2 = a.scale_log2 * pow2f(-(eq + ek));
         __syncwarp();
 
-        const int tl = T - 1;
-        for (int mt = 0; mt < NP; ++mt) {
-            if (mt * 16 >= T) break;
-            // ---- S = Q K^T for query rows mt*16 .. mt*16+15 (keys padded to NP*16)
-            float sacc[2 * NP][4];
+        for (int mg = 0; mg < n_mt; mg += MG) {
+            // ---- S = Q K^T for query tiles mg, mg+1 (each K fragment loaded once)
+            float sacc[MG][2 * NP][4];
 #pragma unroll
-            for (int nt = 0; nt < 2 * NP; ++nt)
-                sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-            const int qrow = min(mt * 16 + (lane & 15), tl);
+            for (int m = 0; m < MG; ++m)
+#pragma unroll
+                for (int nt = 0; nt < 2 * NP; ++nt)
+                    sacc[m][nt][0] = sacc[m][nt][1] = sacc[m][nt][2] = sacc[m][nt][3] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4(aq + swz(qrow, kk * 2 + (lane >> 4)), a0, a1, a2, a3);
+                uint32_t af[MG][4];
+#pragma unroll
+                for (int m = 0; m < MG; ++m)
+                    ldsm_x4(aq + swz(min((mg + m) * 16 + (lane & 15), tl), kk * 2 + (lane >> 4)),
+                            af[m][0], af[m][1], af[m][2], af[m][3]);
 #pragma unroll
                 for (int np = 0; np < NP; ++np) {
-                    if (np * 16 < T) {
+                    if (np < n_mt) {
                         uint32_t b0, b1, b2, b3;
                         const int krow = min(np * 16 + (lane & 7) + ((lane >> 4) << 3), tl);
                         ldsm_x4(ak + swz(krow, kk * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
-                        mma_f16(sacc[2 * np], a0, a1, a2, a3, b0, b1);
-                        mma_f16(sacc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+#pragma unroll
+                        for (int m = 0; m < MG; ++m) {
+                            mma_f16(sacc[m][2 * np], af[m][0], af[m][1], af[m][2], af[m][3], b0, b1);
+                            mma_f16(sacc[m][2 * np + 1], af[m][0], af[m][1], af[m][2], af[m][3], b2, b3);
+                        }
                     }
                 }
             }
-            // ---- softmax over the T keys (rows g and g+8 of the m-tile)
-            float m0 = -INFINITY, m1 = -INFINITY;
+            // ---- softmax over the T keys; P as bf16 A fragments
+            uint32_t pa[MG][NP][4];
+            float il[MG][2];
 #pragma unroll
-            for (int nt = 0; nt < 2 * NP; ++nt) {
-                const int c0 = nt * 8 + 2 * tq;
-                if (c0 >= T) { sacc[nt][0] = -INFINITY; sacc[nt][2] = -INFINITY; }
-                if (c0 + 1 >= T) { sacc[nt][1] = -INFINITY; sacc[nt][3] = -INFINITY; }
-                m0 = fmax3(m0, sacc[nt][0], sacc[nt][1]);
-                m1 = fmax3(m1, sacc[nt][2], sacc[nt][3]);
-            }
-            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-            m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
-            m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
-            const float nm0 = -m0 * scale_log2, nm1 = -m1 * scale_log2;
-            float l0 = 0.f, l1 = 0.f;
+            for (int m = 0; m < MG; ++m) {
+                float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-            for (int nt = 0; nt < 2 * NP; ++nt) {
-                sacc[nt][0] = ex2(fmaf(sacc[nt][0], scale_log2, nm0));
-                sacc[nt][1] = ex2(fmaf(sacc[nt][1], scale_log2, nm0));
-                sacc[nt][2] = ex2(fmaf(sacc[nt][2], scale_log2, nm1));
-                sacc[nt][3] = ex2(fmaf(sacc[nt][3], scale_log2, nm1));
-                l0 += sacc[nt][0] + sacc[nt][1];
-                l1 += sacc[nt][2] + sacc[nt][3];
-            }
-            l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-            l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-            const float il0 = 1.f / l0, il1 = 1.f / l1;
-            // P as bf16 A fragments, k = key index
-            uint32_t pa[NP][4];
+                for (int nt = 0; nt < 2 * NP; ++nt) {
+                    const int c0 = nt * 8 + 2 * tq;
+                    if (c0 >= T) { sacc[m][nt][0] = -INFINITY; sacc[m][nt][2] = -INFINITY; }
+                    if (c0 + 1 >= T) { sacc[m][nt][1] = -INFINITY; sacc[m][nt][3] = -INFINITY; }
+                    m0 = fmax3(m0, sacc[m][nt][0], sacc[m][nt][1]);
+                    m1 = fmax3(m1, sacc[m][nt][2], sacc[m][nt][3]);
+                }
+                m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+                m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+                m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+                m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
+                const float nm0 = -m0 * scale_log2, nm1 = -m1 * scale_log2;
+                float l0 = 0.f, l1 = 0.f;
 #pragma unroll
-            for (int ks = 0; ks < NP; ++ks) {
-                pa[ks][0] = pack_bf16x2(sacc[2 * ks][0], sacc[2 * ks][1]);
-                pa[ks][1] = pack_bf16x2(sacc[2 * ks][2], sacc[2 * ks][3]);
-                pa[ks][2] = pack_bf16x2(sacc[2 * ks + 1][0], sacc[2 * ks + 1][1]);
-                pa[ks][3] = pack_bf16x2(sacc[2 * ks + 1][2], sacc[2 * ks + 1][3]);
-            }
-            __syncwarp();
-            // ---- O = P V, 64 output columns at a time, staged into this m-tile's Q rows
-#pragma unroll
-            for (int dh = 0; dh < 2; ++dh) {
-                float oacc[8][4];
-#pragma unroll
-                for (int nt = 0; nt < 8; ++nt)
-                    oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
+                for (int nt = 0; nt < 2 * NP; ++nt) {
+                    sacc[m][nt][0] = ex2(fmaf(sacc[m][nt][0], scale_log2, nm0));
+                    sacc[m][nt][1] = ex2(fmaf(sacc[m][nt][1], scale_log2, nm0));
+                    sacc[m][nt][2] = ex2(fmaf(sacc[m][nt][2], scale_log2, nm1));
+                    sacc[m][nt][3] = ex2(fmaf(sacc[m][nt][3], scale_log2, nm1));
+                    l0 += sacc[m][nt][0] + sacc[m][nt][1];
+                    l1 += sacc[m][nt][2] + sacc[m][nt][3];
+                }
+                l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+                l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+                il[m][0] = 1.f / l0;
+                il[m][1] = 1.f / l1;
 #pragma unroll
                 for (int ks = 0; ks < NP; ++ks) {
-                    if (ks * 16 < T) {
+                    pa[m][ks][0] = pack_bf16x2(sacc[m][2 * ks][0], sacc[m][2 * ks][1]);
+                    pa[m][ks][1] = pack_bf16x2(sacc[m][2 * ks][2], sacc[m][2 * ks][3]);
+                    pa[m][ks][2] = pack_bf16x2(sacc[m][2 * ks + 1][0], sacc[m][2 * ks + 1][1]);
+                    pa[m][ks][3] = pack_bf16x2(sacc[m][2 * ks + 1][2], sacc[m][2 * ks + 1][3]);
+                }
+            }
+            // every lane is done reading these Q rows before O overwrites them
+            // (later groups read only higher rows)
+            __syncwarp();
+            // ---- O = P V, 64 output columns at a time, staged into the Q rows as bf16
+#pragma unroll
+            for (int dh = 0; dh < 2; ++dh) {
+                float oacc[MG][8][4];
+#pragma unroll
+                for (int m = 0; m < MG; ++m)
+#pragma unroll
+                    for (int nt = 0; nt < 8; ++nt)
+                        oacc[m][nt][0] = oacc[m][nt][1] = oacc[m][nt][2] = oacc[m][nt][3] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < NP; ++ks) {
+                    if (ks < n_mt) {
                         const int vrow = min(ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), tl);
 #pragma unroll
                         for (int dp = 0; dp < 4; ++dp) {
                             uint32_t b0, b1, b2, b3;
                             ldsm_x4_t(av + swz(vrow, dh * 8 + dp * 2 + (lane >> 4)), b0, b1, b2, b3);
-                            mma_bf16(oacc[2 * dp], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b0, b1);
-                            mma_bf16(oacc[2 * dp + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b2, b3);
+#pragma unroll
+                            for (int m = 0; m < MG; ++m) {
+                                mma_bf16(oacc[m][2 * dp], pa[m][ks][0], pa[m][ks][1], pa[m][ks][2],
+                                         pa[m][ks][3], b0, b1);
+                                mma_bf16(oacc[m][2 * dp + 1], pa[m][ks][0], pa[m][ks][1],
+                                         pa[m][ks][2], pa[m][ks][3], b2, b3);
+                            }
                         }
                     }
                 }
-                const int r0 = mt * 16 + g, r1 = r0 + 8;
 #pragma unroll
-                for (int nt = 0; nt < 8; ++nt) {
-                    const int c = dh * 8 + nt;
-                    if (r0 < T)
-                        *reinterpret_cast<uint32_t *>(sq + swz(r0, c) + 4 * tq) =
-                            pack_bf16x2(oacc[nt][0] * il0, oacc[nt][1] * il0);
-                    if (r1 < T)
-                        *reinterpret_cast<uint32_t *>(sq + swz(r1, c) + 4 * tq) =
-                            pack_bf16x2(oacc[nt][2] * il1, oacc[nt][3] * il1);
+                for (int m = 0; m < MG; ++m) {
+                    const int r0 = (mg + m) * 16 + g, r1 = r0 + 8;
+#pragma unroll
+                    for (int nt = 0; nt < 8; ++nt) {
+                        const int c = dh * 8 + nt;
+                        if (r0 < T)
+                            *reinterpret_cast<uint32_t *>(sq + swz(r0, c) + 4 * tq) =
+                                pack_bf16x2(oacc[m][nt][0] * il[m][0], oacc[m][nt][1] * il[m][0]);
+                        if (r1 < T)
+                            *reinterpret_cast<uint32_t *>(sq + swz(r1, c) + 4 * tq) =
+                                pack_bf16x2(oacc[m][nt][2] * il[m][1], oacc[m][nt][3] * il[m][1]);
+                    }
                 }
             }
         }
         __syncwarp();
-        const size_t base = row0(task);
-        for (int idx = lane; idx < T * 16; idx += 32) {
-            const int r = idx >> 4, c = idx & 15;
-            const uint4 v = *reinterpret_cast<const uint4 *>(sq + swz(r, c));
-            *reinterpret_cast<uint4 *>(a.o + base + r * tstride + c * 8) = v;
-        }
+        for (int r = rlane; r < T; r += 2)
+            *reinterpret_cast<uint4 *>(a.o + base + r * tstride + cch * 8) =
+                *reinterpret_cast<const uint4 *>(sq + swz(r, cch));
         __syncwarp();
     }
 }
