@@ -15,6 +15,13 @@
 //   warp  8     tcgen05.mma issuer (one thread) and TMEM allocator
 //   warp  9     TMA loader (one thread)
 //   warps 10-11 idle (they complete the producer warpgroup for setmaxnreg)
+//
+// Work units (1-D grid): units below n_whole each cover one 256-row tile over
+// all keys of its segment.  When the last wave would leave SMs idle, its tiles
+// are instead covered by two units each, one per half of the key tiles; each
+// half writes its normalised fp32 output with its row maximum and sum to the
+// workspace, and the second half to finish (a per-tile counter) merges the
+// two and writes O.
 // TMEM (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1, 128 columns each;
 // P (bf16 pairs) overwrites the first 64 columns of its S.  The MMA issuer
 // ping-pongs the two query tiles so that one tile's softmax overlaps the
@@ -61,12 +68,15 @@ enum Bar {
     B_PFULL0, B_PFULL1,
     B_OFULL,
     B_DRAIN,
+    B_EPI,        // split units: every softmax thread stored its partial
+    B_EPI_GO,     // split units: the merge decision is published
     NUM_BARS
 };
 
 constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
-constexpr int kSmemUsed = OFF_ABORT + 8;
+constexpr int OFF_MERGE = OFF_ABORT + 8;     // int: this unit merges the two halves
+constexpr int kSmemUsed = OFF_MERGE + 8;
 constexpr int kSmemBytes = kSmemUsed + 1024;   // slack to align the base to 1024 B
 
 constexpr uint32_t kTmemCols = 512;
@@ -83,6 +93,11 @@ struct AttnArgs {
     int N;             // tokens per (batch, head) sequence
     int seg_len;       // tokens per segment (N, or H'W' for the spatial pass)
     int q_blocks;      // 256-row query blocks per segment
+    int n_seg;         // segments per sequence
+    int n_whole;       // units covering a whole tile; the rest are half-key units
+    float *part_o;     // [split tiles][2][256][128] normalised partial outputs
+    float2 *part_ml;   // [split tiles][2][256] (row maximum in log2 units, row sum)
+    int *part_count;   // [split tiles] halves finished
     float scale_log2;  // softmax scale * log2(e)
     int rope_q;        // 1: rotate Q tiles with the table
     const float2 *rope_tab;
@@ -104,6 +119,8 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr) {
 }
 
 // Turn row `r` of a swizzled 128x128 Q tile in shared memory by 3D RoPE.
+// All 64 (cos, sin) pairs of the row are fetched first (read-only loads, all
+// in flight together), then the row is rotated in place.
 __device__ __forceinline__ void rope_q_row(uint8_t *tile, int r, int n, const AttnArgs &a) {
     const RopeParams &rp = a.rp;
     if (n >= rp.n_video) return;   // text token or a padding row past N
@@ -111,6 +128,9 @@ __device__ __forceinline__ void rope_q_row(uint8_t *tile, int r, int n, const At
     const int rem = n - t * rp.HW;
     const int h = rem / rp.W;
     const int w = rem - h * rp.W;
+    float2 cs[64];
+#pragma unroll
+    for (int p = 0; p < 64; ++p) cs[p] = __ldg(&a.rope_tab[table_index(rp, p, t, h, w)]);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -119,10 +139,10 @@ __device__ __forceinline__ void rope_q_row(uint8_t *tile, int r, int n, const At
                                                    ((c ^ (r & 7)) << 4));
             uint4 v = *ptr;
             const int p0 = half * 32 + c * 4;
-            v.x = rotate_pair(v.x, a.rope_tab[table_index(rp, p0 + 0, t, h, w)]);
-            v.y = rotate_pair(v.y, a.rope_tab[table_index(rp, p0 + 1, t, h, w)]);
-            v.z = rotate_pair(v.z, a.rope_tab[table_index(rp, p0 + 2, t, h, w)]);
-            v.w = rotate_pair(v.w, a.rope_tab[table_index(rp, p0 + 3, t, h, w)]);
+            v.x = rotate_pair(v.x, cs[p0 + 0]);
+            v.y = rotate_pair(v.y, cs[p0 + 1]);
+            v.z = rotate_pair(v.z, cs[p0 + 2]);
+            v.w = rotate_pair(v.w, cs[p0 + 3]);
             *ptr = v;
         }
     }
@@ -139,14 +159,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.y;
-    const int seg = blockIdx.x / a.q_blocks;
-    const int qb = blockIdx.x - seg * a.q_blocks;
+    // unit -> tile and key-tile range [j0, j1)
+    const int unit = blockIdx.x;
+    const bool split = unit >= a.n_whole;
+    const int split_idx = split ? (unit - a.n_whole) >> 1 : 0;
+    const int part = split ? (unit - a.n_whole) & 1 : 0;
+    const int tile = split ? a.n_whole + split_idx : unit;
+    const int qb = tile % a.q_blocks;
+    const int seg = (tile / a.q_blocks) % a.n_seg;
+    const int bh = tile / (a.q_blocks * a.n_seg);
     const int seg_start = seg * a.seg_len;
     const int seg_end = seg_start + a.seg_len;
     const int q0 = seg_start + qb * (2 * BM);
-    const int n_kv = (a.seg_len + BN - 1) / BN;
-    const int kv_last_valid = a.seg_len - (n_kv - 1) * BN;
+    const int n_kv_all = (a.seg_len + BN - 1) / BN;
+    const int kv_last_valid = a.seg_len - (n_kv_all - 1) * BN;
+    const int j0 = split && part ? n_kv_all / 2 : 0;
+    const int j1 = split && !part ? n_kv_all / 2 : n_kv_all;
+    const int n_kv = j1 - j0;   // key tiles of this unit; local step jj = j - j0
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_QFULL), 1);
@@ -164,6 +193,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(bar(B_PFULL1), BM);
         mbar_init(bar(B_OFULL), 1);
         mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_EPI), 2 * BM);
+        mbar_init(bar(B_EPI_GO), 1);
         *abort_flag = 0;
         mbar_init_fence();
         fence_proxy_async_smem();
@@ -197,7 +228,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             for (int j = 0; j < n_kv; ++j) {
                 const int s = j & 1;
                 const uint32_t ph = (j >> 1) & 1;
-                const int kv0 = seg_start + j * BN;
+                const int kv0 = seg_start + (j0 + j) * BN;
                 if (j >= kStages &&
                     !(ok = mbar_wait(bar(B_KEMPTY0 + s), ph ^ 1, abort_flag, VA3D_DEVERR_TIMEOUT_LOAD)))
                     break;
@@ -341,7 +372,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
             for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
             float *s = reinterpret_cast<float *>(sr);
-            const bool masked_tile = (j == n_kv - 1) && (kv_last_valid < BN);
+            const bool masked_tile = (j0 + j == n_kv_all - 1) && (kv_last_valid < BN);
             if (masked_tile) {
 #pragma unroll
                 for (int c = 0; c < BN; ++c)
@@ -425,26 +456,84 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const float inv_l = 1.0f / l;
             const bool valid = n < seg_end;
             uint4 *dst = reinterpret_cast<uint4 *>(a.o + (static_cast<size_t>(bh) * a.N + n) * HD);
+            if (!split) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t ov[32];
-                tmem_ld32(taO + 32 * c, ov);
-                tmem_wait_ld();
-                reg_fence32(ov);
-                uint32_t pk[16];
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(taO + 32 * c, ov);
+                    tmem_wait_ld();
+                    reg_fence32(ov);
+                    uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l,
-                                        __uint_as_float(ov[2 * e + 1]) * inv_l);
-                if (valid) {
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l,
+                                            __uint_as_float(ov[2 * e + 1]) * inv_l);
+                    if (valid) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
-                                                    pk[4 * e + 3]);
+                        for (int e = 0; e < 4; ++e)
+                            dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
+                                                        pk[4 * e + 3]);
+                    }
+                }
+                if (a.lse != nullptr && valid)
+                    a.lse[static_cast<size_t>(bh) * a.N + n] = (m_ref + log2f(l)) * 0.69314718055994531f;
+            } else {
+                // half of the keys: store the normalised partial and its (max, sum)
+                const size_t prow = (static_cast<size_t>(split_idx) * 2 + part) * (2 * BM) + g * BM + r;
+                float4 *po = reinterpret_cast<float4 *>(a.part_o + prow * HD);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(taO + 32 * c, ov);
+                    tmem_wait_ld();
+                    reg_fence32(ov);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        po[c * 8 + e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
+                                                    __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                                    __uint_as_float(ov[4 * e + 2]) * inv_l,
+                                                    __uint_as_float(ov[4 * e + 3]) * inv_l);
+                }
+                a.part_ml[prow] = make_float2(m_ref, l);
+                __threadfence();
+                mbar_arrive(bar(B_EPI));
+                volatile int *merge = reinterpret_cast<volatile int *>(smem + OFF_MERGE);
+                if (threadIdx.x == 0) {
+                    // all 256 rows of this half are stored and fenced: count it
+                    ok = mbar_wait(bar(B_EPI), 0, abort_flag, VA3D_DEVERR_TIMEOUT_SOFTMAX);
+                    *merge = ok ? atomicAdd(&a.part_count[split_idx], 1) : 0;
+                    __threadfence();
+                    mbar_arrive(bar(B_EPI_GO));
+                }
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_EPI_GO), 0, abort_flag,
+                                                       VA3D_DEVERR_TIMEOUT_SOFTMAX));
+                if (ok && *merge == 1) {
+                    // the other half finished first: merge both and write O
+                    __threadfence();
+                    const size_t orow = (static_cast<size_t>(split_idx) * 2 + (1 - part)) * (2 * BM) + g * BM + r;
+                    const float2 ml_o = __ldcg(&a.part_ml[orow]);
+                    const float m_max = fmaxf(m_ref, ml_o.x);
+                    const float w_s = l * ex2(m_ref - m_max);
+                    const float w_o = ml_o.y * ex2(ml_o.x - m_max);
+                    const float inv_w = 1.0f / (w_s + w_o);
+                    const float c_s = w_s * inv_w, c_o = w_o * inv_w;
+                    const float4 *pa = reinterpret_cast<const float4 *>(a.part_o + prow * HD);
+                    const float4 *pb = reinterpret_cast<const float4 *>(a.part_o + orow * HD);
+#pragma unroll 4
+                    for (int c = 0; c < 16; ++c) {
+                        const float4 x0 = __ldcg(pa + 2 * c), x1 = __ldcg(pa + 2 * c + 1);
+                        const float4 y0 = __ldcg(pb + 2 * c), y1 = __ldcg(pb + 2 * c + 1);
+                        if (valid)
+                            dst[c] = make_uint4(pack_bf16x2(x0.x * c_s + y0.x * c_o, x0.y * c_s + y0.y * c_o),
+                                                pack_bf16x2(x0.z * c_s + y0.z * c_o, x0.w * c_s + y0.w * c_o),
+                                                pack_bf16x2(x1.x * c_s + y1.x * c_o, x1.y * c_s + y1.y * c_o),
+                                                pack_bf16x2(x1.z * c_s + y1.z * c_o, x1.w * c_s + y1.w * c_o));
+                    }
+                    if (a.lse != nullptr && valid)
+                        a.lse[static_cast<size_t>(bh) * a.N + n] =
+                            (m_max + log2f(w_s + w_o)) * 0.69314718055994531f;
                 }
             }
-            if (a.lse != nullptr && valid)
-                a.lse[static_cast<size_t>(bh) * a.N + n] = (m_ref + log2f(l)) * 0.69314718055994531f;
         }
     }
 

@@ -54,7 +54,12 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t packed, float2 cs) {
 
 // Build the cos/sin table for a grid: entries (t, j) at t*half_t + j, then
 // (h, j) at tab_h + h*half_h + j, then (w, j) at tab_w + w*half_w + j.
-__global__ void rope_table_kernel(float2 *__restrict__ tab, const __grid_constant__ RopeParams rp) {
+// It also clears `n_zero` ints at `zero` (per-call counters of the attention
+// kernel that follows on the same stream).
+__global__ void rope_table_kernel(float2 *__restrict__ tab, int *__restrict__ zero, int n_zero,
+                                  const __grid_constant__ RopeParams rp) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n_zero; e += gridDim.x * blockDim.x)
+        zero[e] = 0;
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < rp.tab_entries;
          e += gridDim.x * blockDim.x) {
         int p, pos;

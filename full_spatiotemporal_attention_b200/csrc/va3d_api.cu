@@ -71,6 +71,22 @@ size_t tensor_bytes(int B, int heads, int N) {
     return static_cast<size_t>(B) * heads * N * kHeadDim * 2;
 }
 
+// Scratch for tiles of the last wave split over two key halves: per tile two
+// normalised fp32 partial outputs of 256 rows, their (max, sum) and a counter.
+// At most kMaxSplit tiles are split (half of the SMs of a GPU with up to 256).
+constexpr int kMaxSplit = 128;
+constexpr size_t kSplitOBytes = 2 * 256 * 128 * 4;
+constexpr size_t kSplitMLBytes = 2 * 256 * 8;
+
+long long attn_tiles(int BH, int N) {
+    return static_cast<long long>(BH) * ((N + 255) / 256);
+}
+
+size_t split_bytes_for(long long tiles) {
+    const long long n = std::min<long long>(kMaxSplit, tiles);
+    return round_up(static_cast<size_t>(n) * (kSplitOBytes + kSplitMLBytes + 4), 256);
+}
+
 RopeParams make_rope_params(const va3d_grid_t *g) {
     RopeParams rp;
     std::memset(&rp, 0, sizeof rp);
@@ -131,11 +147,12 @@ int launch_status() {
     return cudaGetLastError() == cudaSuccess ? VA3D_OK : VA3D_ERR_CUDA;
 }
 
-int launch_table(float2 *tab, const RopeParams &rp, cudaStream_t st) {
-    if (rp.tab_entries == 0) return VA3D_OK;
+int launch_table(float2 *tab, int *zero, int n_zero, const RopeParams &rp, cudaStream_t st) {
+    const int work = std::max(rp.tab_entries, n_zero);
+    if (work == 0) return VA3D_OK;
     const int threads = 256;
-    const int blocks = (rp.tab_entries + threads - 1) / threads;
-    rope_table_kernel<<<blocks, threads, 0, st>>>(tab, rp);
+    const int blocks = (work + threads - 1) / threads;
+    rope_table_kernel<<<blocks, threads, 0, st>>>(tab, zero, n_zero, rp);
     return launch_status();
 }
 
@@ -148,9 +165,29 @@ int launch_rope(const void *x, void *y, int BH, int N, const RopeParams &rp, cud
 }
 
 // Attention over segments of seg_len tokens (n_seg * seg_len == n_video or N).
+// Split scratch region: kMaxSplit partial outputs, then (max, sum) pairs,
+// then counters (cleared by the table kernel before every launch).
+struct SplitScratch {
+    float *part_o;
+    float2 *part_ml;
+    int *count;
+    int capacity;   // tiles that fit
+};
+
+SplitScratch split_scratch(void *base, size_t bytes) {
+    SplitScratch sc;
+    const size_t per = kSplitOBytes + kSplitMLBytes + 4;
+    sc.capacity = base == nullptr ? 0 : static_cast<int>(std::min<size_t>(kMaxSplit, bytes / per));
+    uint8_t *p = static_cast<uint8_t *>(base);
+    sc.part_o = reinterpret_cast<float *>(p);
+    sc.part_ml = reinterpret_cast<float2 *>(p + sc.capacity * kSplitOBytes);
+    sc.count = reinterpret_cast<int *>(p + sc.capacity * (kSplitOBytes + kSplitMLBytes));
+    return sc;
+}
+
 int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float *lse, int BH, int N,
                 int seg_len, int n_seg, const RopeParams &rp, const float2 *tab, float scale,
-                cudaStream_t st) {
+                const SplitScratch &sc, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     int rc;
     if ((rc = make_map(&mq, q, N, BH, fa::BM)) != VA3D_OK) return rc;
@@ -167,13 +204,29 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
     a.o = static_cast<__nv_bfloat16 *>(o);
     a.lse = lse;
     a.rp = rp;
+    a.n_seg = n_seg;
+    // One CTA per SM.  If the last wave of tiles would fill at most half of the
+    // SMs and every tile has at least two 128-key steps, each of its tiles is
+    // covered by two units over half of the keys instead.
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return VA3D_ERR_CUDA;
+    const long long tiles = static_cast<long long>(BH) * n_seg * a.q_blocks;
+    const long long tail = sms > 0 ? tiles % sms : 0;
+    const int n_kv = (seg_len + fa::BN - 1) / fa::BN;
+    long long split = 0;
+    if (tail > 0 && 2 * tail <= sms && tail <= sc.capacity && n_kv >= 2) split = tail;
+    a.n_whole = static_cast<int>(tiles - split);
+    a.part_o = sc.part_o;
+    a.part_ml = sc.part_ml;
+    a.part_count = sc.count;
     if (cudaFuncSetAttribute(fa::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::kSmemBytes) != cudaSuccess)
         return VA3D_ERR_CUDA;
-    const long long gx = static_cast<long long>(n_seg) * a.q_blocks;
-    if (gx > 0x7fffffffll) return VA3D_ERR_UNSUPPORTED;
-    dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(BH));
-    fa::attn_fwd_kernel<<<grid, fa::kThreads, fa::kSmemBytes, st>>>(mq, mk, mv, a);
+    const long long units = tiles + split;
+    if (units > 0x7fffffffll) return VA3D_ERR_UNSUPPORTED;
+    fa::attn_fwd_kernel<<<static_cast<unsigned>(units), fa::kThreads, fa::kSmemBytes, st>>>(mq, mk, mv, a);
     return launch_status();
 }
 
@@ -229,6 +282,7 @@ struct Prepared {
     const float2 *tab;
     const void *k_rot;
     float scale;
+    SplitScratch split;
 };
 
 int prepare(const void *q, const void *k, const void *v, int B, int heads, int N, int head_dim,
@@ -248,7 +302,13 @@ int prepare(const void *q, const void *k, const void *v, int B, int heads, int N
     out->rp = make_rope_params(grid);
     out->tab = static_cast<const float2 *>(workspace);
     out->scale = softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(double(head_dim)));
-    if ((rc = launch_table(static_cast<float2 *>(workspace), out->rp, st)) != VA3D_OK) return rc;
+    // workspace: [angle table | rotated keys (unless given) | split scratch]
+    size_t used = table_bytes(grid) + ((flags & VA3D_K_ROTATED) ? 0 : tensor_bytes(B, heads, N));
+    out->split = split_scratch(used < workspace_bytes ? static_cast<uint8_t *>(workspace) + used : nullptr,
+                               used < workspace_bytes ? workspace_bytes - used : 0);
+    if ((rc = launch_table(static_cast<float2 *>(workspace), out->split.count, out->split.capacity,
+                           out->rp, st)) != VA3D_OK)
+        return rc;
     if (flags & VA3D_K_ROTATED) {
         out->k_rot = k;
     } else if (!need_k_rot) {
@@ -305,6 +365,7 @@ size_t va3d_workspace_bytes(int B, int heads, int N, int head_dim, const va3d_gr
     if (check_grid(grid, N, head_dim) != VA3D_OK) return 0;
     size_t bytes = table_bytes(grid);
     if (!(flags & VA3D_K_ROTATED)) bytes += tensor_bytes(B, heads, N);
+    bytes += split_bytes_for(attn_tiles(B * heads, N));
     return bytes;
 }
 
@@ -331,7 +392,7 @@ int attn3d_full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, 
     int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
                      workspace_bytes, true, st, &p);
     if (rc != VA3D_OK) return rc;
-    return launch_attn(q, p.k_rot, v, o, lse, B * heads, N, N, 1, p.rp, p.tab, p.scale, st);
+    return launch_attn(q, p.k_rot, v, o, lse, B * heads, N, N, 1, p.rp, p.tab, p.scale, p.split, st);
 }
 
 int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
@@ -351,7 +412,7 @@ int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 
     if (rc != VA3D_OK) return rc;
     if (o_spatial != nullptr) {
         rc = launch_attn(q, p.k_rot, v, o_spatial, nullptr, B * heads, N, p.rp.HW, p.rp.T, p.rp,
-                         p.tab, p.scale, st);
+                         p.tab, p.scale, p.split, st);
         if (rc != VA3D_OK) return rc;
     }
     if (o_temporal != nullptr)

@@ -73,8 +73,15 @@ def test_workspace_bytes(va):
     g = va.Grid.make(21, 30, 52)
     tab = 8 * (21 * 22 + 30 * 21 + 52 * 21)
     tab = (tab + 255) // 256 * 256
-    assert va.workspace_bytes(1, 12, 32760, g) == tab + 12 * 32760 * 256
-    assert va.workspace_bytes(1, 12, 32760, g, k_rotated=True) == tab
+    # scratch for splitting the last wave's tiles over two key halves: at most
+    # 128 tiles x (two 256x128 fp32 partials + two 256-row (max, sum) + counter)
+    split = (min(128, 12 * 128) * (2 * 256 * 128 * 4 + 2 * 256 * 8 + 4) + 255) // 256 * 256
+    assert va.workspace_bytes(1, 12, 32760, g) == tab + 12 * 32760 * 256 + split
+    assert va.workspace_bytes(1, 12, 32760, g, k_rotated=True) == tab + split
+    tiny = va.Grid.make(2, 4, 4)
+    tab_tiny = (8 * (2 * 22 + 4 * 21 + 4 * 21) + 255) // 256 * 256
+    split_tiny = (2 * (2 * 256 * 128 * 4 + 2 * 256 * 8 + 4) + 255) // 256 * 256
+    assert va.workspace_bytes(1, 2, 32, tiny, k_rotated=True) == tab_tiny + split_tiny
     assert va.workspace_bytes(1, 12, 32761, g) == 0          # N inconsistent with the grid
     bad = va.Grid.make(21, 30, 52, dims=(44, 42, 40))
     assert va.workspace_bytes(1, 12, 32760, bad) == 0
