@@ -143,20 +143,25 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------
 
-def init_dist(args):
+def init_dist(backend="nccl"):
+    """Join the job's process group when launched with WORLD_SIZE > 1 (one
+    process per GPU, rendezvous from the MASTER_* environment).  The CPU
+    tests use backend "gloo", which binds no GPU."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        import torch
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        if backend == "nccl":
+            import torch
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return rank, world, local
 
 
 def max_over_ranks(x, world, device):
+    """The largest of every rank's x (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
@@ -170,6 +175,38 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+REPLICA_SEED_STRIDE = 7919
+
+
+def replica_workload(w, rank):
+    """Rank r's replica: the same shapes with its own seed, so that the ranks
+    of a weak-scaling job attend over independent sequences (rank 0 keeps the
+    workload's own seed, hence the 1-GPU line's inputs)."""
+    import dataclasses
+    return w if rank == 0 else dataclasses.replace(w, seed=w.seed + REPLICA_SEED_STRIDE * rank)
+
+
+def job_tflops(flops_per_rank, world, ms):
+    """Whole-job throughput: every rank's FLOPs over the slowest rank's time."""
+    return world * flops_per_rank / (ms / 1e3) / 1e12
+
+
+def job_config(w, world):
+    return {"workload": w.description, "grid": [w.T, w.H, w.W], "tokens": w.N,
+            "heads": w.heads, "head_dim": HEAD_DIM, "batch": w.batch,
+            "rope_split": list(w.dims), "theta": w.theta,
+            "flops_per_step": full_flops(w), "global_batch": w.batch * world, "seq_len": w.N,
+            "parallelism": f"replicas x{world} (independent sequences, no collective)",
+            "l2": l2_note(w)}
+
+
+def l2_note(w):
+    mb = 4 * w.batch * w.heads * w.N * HEAD_DIM * 2 / 1e6
+    if mb > 126:
+        return f"inputs exceed L2 (Q,K,V,O = {mb:.0f} MB > 126 MB); no flush"
+    return f"inputs fit in L2 (Q,K,V,O = {mb:.1f} MB)"
 
 
 def to_dev(bits, device):
@@ -235,7 +272,7 @@ def bench_ours(args, rank, world, local):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    w = si.WORKLOADS[args.workload]
+    w = replica_workload(si.WORKLOADS[args.workload], rank)
     qb, kb, vb = si.qkv(w)
     q, k, v = (to_dev(x, device) for x in (qb, kb, vb))
     g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
@@ -280,7 +317,7 @@ def bench_ours(args, rank, world, local):
     _, rope_ms = timed_loop(rope_only, max(args.steps, 10), 3, world, device)
 
     flops = full_flops(w)
-    value = world * flops / (step_ms / 1e3) / 1e12
+    value = job_tflops(flops, world, step_ms)
     peak_tf, peak_gbs, peak_src = peaks()
     achieved = flops / (attn_ms / 1e3) / 1e12
     traffic = recorded_traffic("attn_fwd_kernel", w.name)
@@ -315,14 +352,9 @@ def bench_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded splitmix64 + Box-Muller bf16 N(0,1))",
-        "config": {"workload": w.description, "grid": [w.T, w.H, w.W], "tokens": w.N,
-                   "heads": w.heads, "head_dim": HEAD_DIM, "batch": w.batch,
-                   "rope_split": list(w.dims), "theta": w.theta,
-                   "flops_per_step": flops, "global_batch": w.batch * world, "seq_len": w.N,
-                   "parallelism": f"replicas x{world} (independent sequences, no collective)",
-                   "l2": "inputs exceed L2 (Q,K,V,O = 403 MB > 126 MB); no flush"},
+        "config": job_config(w, world),
         "pct_of_peak": round(100.0 * value / world / peak_tf, 2),
-        "e2e": {"value": round(world * flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_tflops(flops, world, e2e_ms), 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes},
         "gpu_launches": 3 * args.steps,
@@ -434,7 +466,7 @@ def bench_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.description, "tokens": w.N, "heads": w.heads},
+        "config": job_config(w, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -453,7 +485,7 @@ def main():
         if rank == 0:
             print(json.dumps(bench_reference(args, rank, world)), flush=True)
         return
-    rank, world, local = init_dist(args)
+    rank, world, local = init_dist("nccl")
     line = bench_ours(args, rank, world, local)
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -7,7 +7,6 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 
 #include "va3d.h"
 
@@ -228,15 +227,6 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
                    "+r"(r[30]), "+r"(r[31]));
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-
 // ----------------------------------------------------- UMMA descriptors
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 layout version 1.
@@ -307,19 +297,6 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
-}
-
-// 2^x for a pair with one MUFU operation: x is rounded to fp16 and both
-// exponentials come from the unit's packed fp16 form.  Used where x <= 8 (so
-// 2^x <= 256 fits fp16) and the result is rounded to bf16 anyway: rounding x
-// to fp16 perturbs 2^x by at most 2^-11 * |x| * ln 2 relative, below bf16's
-// 2^-9 for |x| < 4 and comparable to it up to |x| = 8.
-__device__ __forceinline__ float2 exp2_f16x2(float2 x) {
-    uint32_t h, e;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x.y), "f"(x.x));
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-    __half2 r = *reinterpret_cast<__half2 *>(&e);
-    return __half22float2(r);
 }
 
 // 2^x for a pair on the FMA pipe instead of the MUFU unit.  Range reduction
