@@ -160,6 +160,11 @@ def _load():
                                             ctypes.POINTER(ctypes.c_int),
                                             ctypes.POINTER(ctypes.c_int)]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_cross_attention.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_long, ctypes.c_long, ctypes.c_long,
+                                               ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
+                                               ctypes.c_long, ctypes.c_void_p, ctypes.c_void_p]
+        lib.oracle_cross_attention.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -220,6 +225,30 @@ def attention(q_bits, k_bits, v_bits, grid: Grid, mode="full", rows=None, scale=
                                   lse.ctypes.data if want_lse else None)
     if rc != 0:
         raise ValueError(f"oracle_attention rejected the arguments ({rc})")
+    return (out, lse) if want_lse else out
+
+
+def cross_attention(q_bits, k_bits, v_bits, rows=None, scale=None, want_lse=False):
+    """fp64 text cross-attention of a Wan block ("04 HunyuanVideo and Wan",
+    section 3.1): query rows of q [..., Nq, d] attend to all keys of
+    k, v [..., Nkv, d]; no rotation.  Returns out [BH, len(rows), d] (and lse)."""
+    q, k, v = _bits(q_bits), _bits(k_bits), _bits(v_bits)
+    Nq, D = q.shape[-2], q.shape[-1]
+    Nkv = k.shape[-2]
+    BH = int(np.prod(q.shape[:-2])) if q.ndim > 2 else 1
+    if k.shape != v.shape or k.shape[-1] != D or int(np.prod(k.shape[:-2])) != BH:
+        raise ValueError("k and v must be [..., Nkv, d] with q's leading dims")
+    if rows is None:
+        rows = np.arange(Nq, dtype=np.int64)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.empty((BH, rows.size, D), dtype=np.float64)
+    lse = np.empty((BH, rows.size), dtype=np.float64) if want_lse else None
+    rc = _load().oracle_cross_attention(q.ctypes.data, k.ctypes.data, v.ctypes.data, BH, Nq, Nkv,
+                                        D, float(scale) if scale else 0.0, rows.ctypes.data,
+                                        rows.size, out.ctypes.data,
+                                        lse.ctypes.data if want_lse else None)
+    if rc != 0:
+        raise ValueError(f"oracle_cross_attention rejected the arguments ({rc})")
     return (out, lse) if want_lse else out
 
 

@@ -21,7 +21,9 @@
  *    128 dims into 22/21/21 rotary pairs (axes_dim = [44, 42, 42]).
  *  - "04 HunyuanVideo and Wan" (note.shouss.top), section 2.5: head dim 128,
  *    RoPE split (16, 56, 56); sections 2.3/2.4: joint attention over the
- *    concatenated video+text sequence.
+ *    concatenated video+text sequence; section 3.1: a Wan block's text
+ *    cross-attention (queries from the video tokens, keys and values from
+ *    the text encoder's tokens, which the step does not update).
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - pairs are adjacent (2j, 2j+1) inside each axis range;
@@ -278,5 +280,62 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     }
     free(kr);
     free(vd);
+    return ORACLE_OK;
+}
+
+/*
+ * Text cross-attention of a Wan block ("04 HunyuanVideo and Wan", section
+ * 3.1): every video query row attends to all Nkv text keys; neither side is
+ * rotated (the 3D positions belong to the video self-attention).  Same
+ * arithmetic as oracle_attention: s_j = scale * q.k_j, m = max s_j,
+ * o = sum exp(s_j - m) v_j / sum exp(s_j - m), lse = m + log(sum).
+ * q is [BH, Nq, D], k and v are [BH, Nkv, D] bf16 bits; rows index q.
+ */
+int oracle_cross_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           long BH, long Nq, long Nkv, int head_dim, double scale,
+                           const long *rows, long nrows, double *out, double *lse)
+{
+    if (BH < 1 || Nq < 1 || Nkv < 1 || head_dim < 1) return ORACLE_EINVAL;
+    for (long r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= Nq) return ORACLE_EINVAL;
+    if (!(scale > 0.0)) scale = 1.0 / sqrt((double)head_dim);
+    const size_t D = (size_t)head_dim;
+
+#pragma omp parallel
+    {
+        double *qx = (double *)malloc(sizeof(double) * D);
+        double *s = (double *)malloc(sizeof(double) * (size_t)Nkv);
+        double *acc = (double *)malloc(sizeof(double) * D);
+#pragma omp for schedule(dynamic, 16) collapse(2)
+        for (long bh = 0; bh < BH; ++bh) {
+            for (long r = 0; r < nrows; ++r) {
+                const uint16_t *qb = q + ((size_t)bh * Nq + rows[r]) * D;
+                const uint16_t *kb = k + (size_t)bh * Nkv * D;
+                const uint16_t *vb = v + (size_t)bh * Nkv * D;
+                for (size_t c = 0; c < D; ++c) qx[c] = bf16_bits_to_double(qb[c]);
+                double m = -INFINITY;
+                for (long j = 0; j < Nkv; ++j) {
+                    double dot = 0.0;
+                    for (size_t c = 0; c < D; ++c)
+                        dot += qx[c] * bf16_bits_to_double(kb[j * D + c]);
+                    s[j] = dot * scale;
+                    if (s[j] > m) m = s[j];
+                }
+                double z = 0.0;
+                for (size_t c = 0; c < D; ++c) acc[c] = 0.0;
+                for (long j = 0; j < Nkv; ++j) {
+                    double p = exp(s[j] - m);
+                    z += p;
+                    for (size_t c = 0; c < D; ++c) acc[c] += p * bf16_bits_to_double(vb[j * D + c]);
+                }
+                double *o = out + ((size_t)bh * nrows + r) * D;
+                for (size_t c = 0; c < D; ++c) o[c] = acc[c] / z;
+                if (lse) lse[bh * nrows + r] = m + log(z);
+            }
+        }
+        free(qx);
+        free(s);
+        free(acc);
+    }
     return ORACLE_OK;
 }

@@ -51,6 +51,7 @@ class Workload:
     seed: int = 1000
     sharpen_frac: float = 0.0   # fraction of tokens whose K is scaled by 2
     description: str = ""
+    n_kv: int = 0               # > 0: cross-attention to n_kv separate key/value tokens
 
     @property
     def n_video(self):
@@ -63,6 +64,11 @@ class Workload:
     @property
     def shape(self):
         return (self.batch, self.heads, self.N, self.head_dim)
+
+    @property
+    def kv_shape(self):
+        n = self.n_kv if self.n_kv > 0 else self.N
+        return (self.batch, self.heads, n, self.head_dim)
 
 
 WORKLOADS = {
@@ -78,6 +84,13 @@ WORKLOADS = {
     "joint720": Workload("joint720", 33, 45, 80, 24, (16, 56, 56), n_text=256, seed=1005,
                          description="129-frame 720x1280 clip, 33x45x80 = 118,800 video tokens "
                                      "+ 256 text tokens, 24 heads"),
+    "cross720": Workload("cross720", 21, 45, 80, 40, (44, 42, 42), seed=1007, n_kv=512,
+                         description="text cross-attention: 21x45x80 = 75,600 video queries "
+                                     "x 512 text keys, 40 heads"),
+    "refimg720": Workload("refimg720", 21, 45, 80, 40, (44, 42, 42), n_text=3 * 4096, seed=1006,
+                          description="81-frame 720x1280 clip, 21x45x80 = 75,600 video tokens "
+                                      "+ 3 reference images x 4,096 tokens = 87,888 tokens, "
+                                      "40 heads"),
 }
 
 
@@ -123,14 +136,15 @@ def sharpened_tokens(w: Workload):
     """Boolean mask over token indices whose K rows are doubled (shared by heads)."""
     if w.sharpen_frac <= 0:
         return np.zeros(w.N, dtype=bool)
-    return uniform(w.seed, SHARPEN_STREAM, w.N) < w.sharpen_frac
+    return uniform(w.seed, SHARPEN_STREAM, w.kv_shape[2]) < w.sharpen_frac
 
 
 def qkv(w: Workload):
-    """(q, k, v) as uint16 bf16 bits shaped [B, heads, N, head_dim]."""
+    """(q, k, v) as uint16 bf16 bits: q [B, heads, N, head_dim], k and v
+    [B, heads, N or n_kv, head_dim]."""
     q = normal_bf16(w.seed, Q_STREAM, w.shape)
-    k = normal_bf16(w.seed, K_STREAM, w.shape)
-    v = normal_bf16(w.seed, V_STREAM, w.shape)
+    k = normal_bf16(w.seed, K_STREAM, w.kv_shape)
+    v = normal_bf16(w.seed, V_STREAM, w.kv_shape)
     sel = sharpened_tokens(w)
     if sel.any():
         # doubling is exact in bf16: add one to the exponent field of nonzero finite values

@@ -140,6 +140,10 @@ def test_page_arithmetic(golden_dir):
     assert round((n720 / n480) ** 2, 1) == vals["attention_growth"][0]
     seq = n720 + 3 * int(vals["reference_image_tokens"][0])
     assert seq == vals["sequence_with_3_refs"][0]
+    # the reference-image workload is that request's shape
+    import seeded_inputs as si
+    ref_w = si.WORKLOADS["refimg720"]
+    assert ref_w.n_video == n720 and ref_w.N == vals["sequence_with_3_refs"][0]
     assert round(((seq / n720) ** 2 - 1) * 100) == vals["attention_cost_rise_percent"][0]
     # the diffusers DiT example: 3 latent frames of 8x8, patch 2, plus 4 text tokens
     lt, lhw = int(vals["dit_latent_T"][0]), int(vals["dit_latent_HW"][0])
@@ -431,6 +435,57 @@ def test_oracle_rejects_bad_arguments():
         oracle.attention(x, x, x, g, mode="spatial")     # factorised passes have no text
     with pytest.raises(ValueError):
         oracle.attention(x, x, x, Grid(2, 2, 2))          # N mismatch
+
+
+# ---------------------------------------------------------------------------
+# text cross-attention (Wan block, "04 HunyuanVideo and Wan" section 3.1)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("nq,nkv", [(37, 11), (5, 300), (64, 1)])
+def test_cross_attention_equals_sdpa(nq, nkv):
+    q = _rand_bits((3, nq, 128), 101)
+    k = _rand_bits((3, nkv, 128), 102)
+    v = _rand_bits((3, nkv, 128), 103)
+    o, lse = oracle.cross_attention(q, k, v, want_lse=True)
+    qf, kf, vf = (bf16_bits_to_f64(x) for x in (q, k, v))
+    np.testing.assert_allclose(o, _sdpa(qf, kf, vf), atol=1e-12, rtol=0)
+    s = torch.from_numpy(qf @ kf.transpose(0, 2, 1) / math.sqrt(128))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), atol=1e-12, rtol=0)
+
+
+def test_cross_attention_special_cases():
+    q = _rand_bits((2, 9, 128), 111, scale=3.0)
+    k = _rand_bits((2, 1, 128), 112)
+    v = _rand_bits((2, 1, 128), 113)
+    # one key: every query copies its value
+    o = oracle.cross_attention(q, k, v)
+    np.testing.assert_array_equal(o, np.broadcast_to(bf16_bits_to_f64(v), o.shape))
+    # zero queries average the values; permuting the keys (with their values)
+    # changes nothing
+    k = _rand_bits((2, 40, 128), 114)
+    v = _rand_bits((2, 40, 128), 115)
+    z = np.zeros((2, 4, 128), dtype=np.uint16)
+    o = oracle.cross_attention(z, k, v)
+    np.testing.assert_allclose(o, np.broadcast_to(bf16_bits_to_f64(v).mean(axis=1, keepdims=True),
+                                                  o.shape), atol=1e-14, rtol=0)
+    perm = np.random.default_rng(0).permutation(40)
+    q = _rand_bits((2, 4, 128), 116)
+    np.testing.assert_allclose(oracle.cross_attention(q, k[:, perm], v[:, perm]),
+                               oracle.cross_attention(q, k, v), atol=1e-14, rtol=0)
+
+
+def test_cross_attention_rows_and_self_attention_consistent():
+    # with keys = the queries' own sequence and no rotation it is the
+    # unrotated full attention
+    g = Grid(2, 3, 5)
+    q, k, v = (_rand_bits((2, g.N, 128), s) for s in (121, 122, 123))
+    full = oracle.attention(q, k, v, g, rotate=False)
+    np.testing.assert_allclose(oracle.cross_attention(q, k, v), full, atol=1e-13, rtol=0)
+    rows = np.array([0, 7, g.N - 1])
+    np.testing.assert_array_equal(oracle.cross_attention(q, k, v, rows=rows),
+                                  oracle.cross_attention(q, k, v)[:, rows])
+    with pytest.raises(ValueError):
+        oracle.cross_attention(q, k, v, rows=np.array([g.N]))
 
 
 # ---------------------------------------------------------------------------
