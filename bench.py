@@ -394,6 +394,30 @@ def extras(va, device, stream, peak_tf, peak_gbs):
             return a, b
         return run
 
+    # the 17-frame clip: full vs factorised cost ratio at 7,800 tokens
+    w = si.WORKLOADS["c17f480"]
+    q, k, v = (to_dev(x, device) for x in si.qkv(w))
+    g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    kr = va.rope3d_apply(k, g)
+    o = torch.empty_like(q)
+    o2 = torch.empty_like(q)
+    ws = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g, k_rotated=True),
+                     dtype=torch.uint8, device=device)
+    _, s_full = timed_loop(ev_pair(lambda: va.attn3d_full_fwd(q, kr, v, g, k_rotated=True, out=o,
+                                                               workspace=ws)), 20, 3, 1, device)
+    _, s_fact = timed_loop(ev_pair(lambda: va.attn_factorized_fwd(
+        q, kr, v, g, k_rotated=True, out_spatial=o, out_temporal=o2, workspace=ws)), 20, 3, 1, device)
+    f_full = 4.0 * w.N ** 2 * HEAD_DIM * w.heads
+    hw = w.H * w.W
+    f_fact = 4.0 * HEAD_DIM * w.heads * (w.T * hw * hw + hw * w.T ** 2)
+    out["c17f480"] = {"tokens": w.N, "heads": w.heads, "full_ms": round(s_full, 4),
+                      "full_tflops": round(f_full / s_full / 1e9, 1),
+                      "factorised_ms": round(s_fact, 4),
+                      "full_over_factorised_time": round(s_full / s_fact, 2),
+                      "full_over_factorised_flops": round(f_full / f_fact, 2)}
+    del q, k, v, kr, o, o2, ws
+    torch.cuda.empty_cache()
+
     w = si.WORKLOADS["c81f720"]
     q, k, v = (to_dev(x, device) for x in si.qkv(w))
     g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
@@ -424,20 +448,46 @@ def extras(va, device, stream, peak_tf, peak_gbs):
     del q, k, v, kr, o, o2, ws
     torch.cuda.empty_cache()
 
-    w = si.WORKLOADS["joint720"]
+    def full_only(name):
+        w = si.WORKLOADS[name]
+        q, k, v = (to_dev(x, device) for x in si.qkv(w))
+        g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+        kr = va.rope3d_apply(k, g)
+        o = torch.empty_like(q)
+        ws = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g, k_rotated=True),
+                         dtype=torch.uint8, device=device)
+        _, ms = timed_loop(ev_pair(lambda: va.attn3d_full_fwd(q, kr, v, g, k_rotated=True, out=o,
+                                                               workspace=ws)), 3, 2, 1, device)
+        del q, k, v, kr, o, ws
+        torch.cuda.empty_cache()
+        f = 4.0 * w.N ** 2 * HEAD_DIM * w.heads
+        return {"tokens": w.N, "heads": w.heads, "ms": round(ms, 3),
+                "tflops": round(f / ms / 1e9, 1), "frac_of_peak": round(f / ms / 1e9 / peak_tf, 4)}
+
+    out["joint720"] = full_only("joint720")
+    # three reference images appended to the 720p clip: the same 40 heads,
+    # 87,888 tokens, so the time should grow like N^2 (x1.35)
+    ref = full_only("refimg720")
+    ref["over_c81f720_time"] = round(ref["ms"] / full_ms, 3)
+    ref["over_c81f720_flops"] = round((ref["tokens"] / w.N) ** 2, 3)
+    out["refimg720"] = ref
+
+    # Wan text cross-attention: 75,600 video queries x 512 text keys, no RoPE
+    w = si.WORKLOADS["cross720"]
     q, k, v = (to_dev(x, device) for x in si.qkv(w))
-    g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
-    kr = va.rope3d_apply(k, g)
     o = torch.empty_like(q)
-    ws = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g, k_rotated=True),
-                     dtype=torch.uint8, device=device)
-    _, j_ms = timed_loop(ev_pair(lambda: va.attn3d_full_fwd(q, kr, v, g, k_rotated=True, out=o,
-                                                            workspace=ws)), 3, 2, 1, device)
-    f_j = 4.0 * w.N ** 2 * HEAD_DIM * w.heads
-    out["joint720"] = {"tokens": w.N, "heads": w.heads, "ms": round(j_ms, 3),
-                       "tflops": round(f_j / j_ms / 1e9, 1),
-                       "frac_of_peak": round(f_j / j_ms / 1e9 / peak_tf, 4)}
-    del q, k, v, kr, o, ws
+    ws = torch.empty(va.cross_workspace_bytes(w.batch, w.heads, w.N, w.n_kv), dtype=torch.uint8,
+                     device=device)
+    _, x_ms = timed_loop(ev_pair(lambda: va.attn_cross_fwd(q, k, v, out=o, workspace=ws)), 10, 3, 1,
+                         device)
+    f_x = 4.0 * w.N * w.n_kv * HEAD_DIM * w.heads
+    b_x = 2 * (2 * w.N + 2 * w.n_kv) * HEAD_DIM * w.heads   # read Q, K, V; write O
+    out["cross720"] = {"queries": w.N, "keys": w.n_kv, "heads": w.heads, "ms": round(x_ms, 4),
+                       "tflops": round(f_x / x_ms / 1e9, 1),
+                       "frac_of_peak": round(f_x / x_ms / 1e9 / peak_tf, 4),
+                       "gbs": round(b_x / x_ms / 1e6, 1),
+                       "frac_of_hbm": round(b_x / x_ms / 1e6 / peak_gbs, 4)}
+    del q, k, v, o, ws
     torch.cuda.empty_cache()
     return out
 

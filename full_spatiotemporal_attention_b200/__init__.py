@@ -11,6 +11,7 @@ Entry points (same names as the C ABI):
 * ``rope3d_apply(x, grid)``                 3D RoPE of a [B, heads, N, 128] tensor
 * ``attn3d_full_fwd(q, k, v, grid)``        full 3D (or joint video+text) attention
 * ``attn_factorized_fwd(q, k, v, grid)``    spatial and temporal passes
+* ``attn_cross_fwd(q, k, v)``               video-to-text cross-attention (no RoPE)
 * ``grid_from_video(frames, height, width)``  token grid of a clip
 * ``workspace_bytes(...)``, ``device_error()``
 """
@@ -28,7 +29,8 @@ HEAD_DIM = 128
 
 SYMBOLS = ("va3d_status_string", "va3d_version", "va3d_grid_from_video",
            "va3d_workspace_bytes", "rope3d_apply", "attn3d_full_fwd",
-           "attn_factorized_fwd", "va3d_device_error", "attn3d_full_fwd_noalloc")
+           "attn_factorized_fwd", "va3d_device_error", "attn3d_full_fwd_noalloc",
+           "va3d_cross_workspace_bytes", "attn_cross_fwd")
 
 
 class VA3DError(RuntimeError):
@@ -80,6 +82,9 @@ def _load():
     lib.attn_factorized_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp, sz, vp]
     lib.va3d_device_error.argtypes = [i]
     lib.attn3d_full_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp]
+    lib.va3d_cross_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.va3d_cross_workspace_bytes.restype = sz
+    lib.attn_cross_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
     return lib
 
 
@@ -242,6 +247,42 @@ def attn_factorized_fwd(q, k, v, grid, *, spatial=True, temporal=True, scale=Non
     if rc != VA3D_OK:
         raise VA3DError("attn_factorized_fwd", rc)
     return out_spatial, out_temporal
+
+
+def cross_workspace_bytes(B, heads, Nq, Nkv):
+    return int(lib.va3d_cross_workspace_bytes(B, heads, Nq, Nkv, HEAD_DIM))
+
+
+def attn_cross_fwd(q, k, v, *, scale=None, return_lse=False, out=None, lse=None,
+                   workspace=None):
+    """Cross-attention of video queries q [B, heads, Nq, 128] to text keys and
+    values k, v [B, heads, Nkv, 128]; no RoPE.  Returns o [B, heads, Nq, 128]
+    (and lse [B, heads, Nq] fp32 if asked)."""
+    torch = _torch()
+    _check(q, "q")
+    _check(k, "k")
+    B, H, Nq, D = q.shape
+    Nkv = k.shape[2]
+    if k.shape[:2] != q.shape[:2]:
+        raise ValueError(f"k has shape {tuple(k.shape)}, expected [{B}, {H}, Nkv, {D}]")
+    _check(v, "v", k.shape)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq)
+                            or not lse.is_contiguous() or not lse.is_cuda):
+        raise ValueError("lse must be a contiguous CUDA float32 [B, heads, Nq] tensor")
+    if workspace is None:
+        workspace = torch.empty(max(cross_workspace_bytes(B, H, Nq, Nkv), 256),
+                                dtype=torch.uint8, device=q.device)
+    rc = lib.attn_cross_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Nq, Nkv, D,
+                            float(scale or 0.0), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(q))
+    if rc != VA3D_OK:
+        raise VA3DError("attn_cross_fwd", rc)
+    return (out, lse) if (return_lse or lse is not None) else out
 
 
 def device_error(reset=True):

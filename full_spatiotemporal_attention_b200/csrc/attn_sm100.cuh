@@ -90,8 +90,10 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int kPolyEvery = 4;
 
 struct AttnArgs {
-    int N;             // tokens per (batch, head) sequence
-    int seg_len;       // tokens per segment (N, or H'W' for the spatial pass)
+    int N;             // query tokens per (batch, head) sequence
+    int seg_len;       // query tokens per segment (N, or H'W' for the spatial pass)
+    int kv_len;        // keys per segment (seg_len for self-attention; segment s's
+                       // keys are rows [s * kv_len, (s + 1) * kv_len) of K and V)
     int q_blocks;      // 256-row query blocks per segment
     int n_seg;         // segments per sequence
     int n_whole;       // units covering a whole tile; the rest are half-key units
@@ -171,8 +173,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int seg_start = seg * a.seg_len;
     const int seg_end = seg_start + a.seg_len;
     const int q0 = seg_start + qb * (2 * BM);
-    const int n_kv_all = (a.seg_len + BN - 1) / BN;
-    const int kv_last_valid = a.seg_len - (n_kv_all - 1) * BN;
+    const int kv_start = seg * a.kv_len;
+    const int n_kv_all = (a.kv_len + BN - 1) / BN;
+    const int kv_last_valid = a.kv_len - (n_kv_all - 1) * BN;
     const int j0 = split && part ? n_kv_all / 2 : 0;
     const int j1 = split && !part ? n_kv_all / 2 : n_kv_all;
     const int n_kv = j1 - j0;   // key tiles of this unit; local step jj = j - j0
@@ -228,7 +231,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             for (int j = 0; j < n_kv; ++j) {
                 const int s = j & 1;
                 const uint32_t ph = (j >> 1) & 1;
-                const int kv0 = seg_start + (j0 + j) * BN;
+                const int kv0 = kv_start + (j0 + j) * BN;
                 if (j >= kStages &&
                     !(ok = mbar_wait(bar(B_KEMPTY0 + s), ph ^ 1, abort_flag, VA3D_DEVERR_TIMEOUT_LOAD)))
                     break;

@@ -185,21 +185,25 @@ SplitScratch split_scratch(void *base, size_t bytes) {
     return sc;
 }
 
+// Q is [BH, N, 128] in n_seg segments of seg_len rows; K and V are
+// [BH, Nkv, 128] in n_seg segments of kv_len rows; segment s of the queries
+// attends to segment s of the keys.
 int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float *lse, int BH, int N,
-                int seg_len, int n_seg, const RopeParams &rp, const float2 *tab, float scale,
-                const SplitScratch &sc, cudaStream_t st) {
+                int Nkv, int seg_len, int kv_len, int n_seg, bool rope_q, const RopeParams &rp,
+                const float2 *tab, float scale, const SplitScratch &sc, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     int rc;
     if ((rc = make_map(&mq, q, N, BH, fa::BM)) != VA3D_OK) return rc;
-    if ((rc = make_map(&mk, k_rot, N, BH, fa::BN)) != VA3D_OK) return rc;
-    if ((rc = make_map(&mv, v, N, BH, fa::BN)) != VA3D_OK) return rc;
+    if ((rc = make_map(&mk, k_rot, Nkv, BH, fa::BN)) != VA3D_OK) return rc;
+    if ((rc = make_map(&mv, v, Nkv, BH, fa::BN)) != VA3D_OK) return rc;
     fa::AttnArgs a;
     std::memset(&a, 0, sizeof a);
     a.N = N;
     a.seg_len = seg_len;
+    a.kv_len = kv_len;
     a.q_blocks = (seg_len + 2 * fa::BM - 1) / (2 * fa::BM);
     a.scale_log2 = static_cast<float>(scale * kLog2e);
-    a.rope_q = 1;
+    a.rope_q = rope_q ? 1 : 0;
     a.rope_tab = tab;
     a.o = static_cast<__nv_bfloat16 *>(o);
     a.lse = lse;
@@ -214,7 +218,7 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
         return VA3D_ERR_CUDA;
     const long long tiles = static_cast<long long>(BH) * n_seg * a.q_blocks;
     const long long tail = sms > 0 ? tiles % sms : 0;
-    const int n_kv = (seg_len + fa::BN - 1) / fa::BN;
+    const int n_kv = (kv_len + fa::BN - 1) / fa::BN;
     long long split = 0;
     if (tail > 0 && 2 * tail <= sms && tail <= sc.capacity && n_kv >= 2) split = tail;
     a.n_whole = static_cast<int>(tiles - split);
@@ -392,7 +396,8 @@ int attn3d_full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, 
     int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
                      workspace_bytes, true, st, &p);
     if (rc != VA3D_OK) return rc;
-    return launch_attn(q, p.k_rot, v, o, lse, B * heads, N, N, 1, p.rp, p.tab, p.scale, p.split, st);
+    return launch_attn(q, p.k_rot, v, o, lse, B * heads, N, N, N, N, 1, true, p.rp, p.tab, p.scale,
+                       p.split, st);
 }
 
 int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
@@ -411,14 +416,46 @@ int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 
                      workspace_bytes, o_spatial != nullptr, st, &p);
     if (rc != VA3D_OK) return rc;
     if (o_spatial != nullptr) {
-        rc = launch_attn(q, p.k_rot, v, o_spatial, nullptr, B * heads, N, p.rp.HW, p.rp.T, p.rp,
-                         p.tab, p.scale, p.split, st);
+        rc = launch_attn(q, p.k_rot, v, o_spatial, nullptr, B * heads, N, N, p.rp.HW, p.rp.HW,
+                         p.rp.T, true, p.rp, p.tab, p.scale, p.split, st);
         if (rc != VA3D_OK) return rc;
     }
     if (o_temporal != nullptr)
         rc = launch_temporal(q, k, (flags & VA3D_K_ROTATED) != 0, v, o_temporal, B * heads, N, p.rp,
                              p.tab, p.scale, st);
     return rc;
+}
+
+size_t va3d_cross_workspace_bytes(int B, int heads, int Nq, int Nkv, int head_dim) {
+    if (check_sizes(B, heads, Nq, head_dim) != VA3D_OK) return 0;
+    if (check_sizes(B, heads, Nkv, head_dim) != VA3D_OK) return 0;
+    return split_bytes_for(attn_tiles(B * heads, Nq));
+}
+
+int attn_cross_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *o,
+                   float *lse, int B, int heads, int Nq, int Nkv, int head_dim, float softmax_scale,
+                   void *workspace, size_t workspace_bytes, void *stream) {
+    int rc;
+    if ((rc = check_sizes(B, heads, Nq, head_dim)) != VA3D_OK) return rc;
+    if ((rc = check_sizes(B, heads, Nkv, head_dim)) != VA3D_OK) return rc;
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return VA3D_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+        (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return VA3D_ERR_ALIGNMENT;
+    if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const float scale =
+        softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(double(head_dim)));
+    // The workspace only holds the scratch for splitting the last wave's
+    // tiles; without one (or with too little) those tiles run whole.
+    SplitScratch sc = split_scratch(workspace, workspace != nullptr ? workspace_bytes : 0);
+    RopeParams none;
+    std::memset(&none, 0, sizeof none);
+    if ((rc = launch_table(nullptr, sc.count, sc.capacity, none, st)) != VA3D_OK) return rc;
+    return launch_attn(q, k, v, o, lse, B * heads, Nq, Nkv, Nq, Nkv, 1, false, none, nullptr, scale,
+                       sc, st);
 }
 
 int va3d_device_error(int reset) {

@@ -16,7 +16,8 @@
  *    attention sees time: factorised or full";
  *  - joint video+text attention: "04 HunyuanVideo and Wan" (note.shouss.top)
  *    sections 2.3-2.4, and the handbook's diffusers example (video tokens +
- *    text tokens attended together in one sequence).
+ *    text tokens attended together in one sequence);
+ *  - text cross-attention: the same page, section 3.1 (Wan's block).
  *
  * Conventions shared by every entry point
  *  - Tensors are contiguous bf16 (bit patterns, va3d_bf16) of shape
@@ -109,7 +110,10 @@ int va3d_grid_from_video(int frames, int height, int width, int d_t, int d_h, in
  * these arguments: a cos/sin table of the grid's rotation angles
  * (8 * (T'*d_t/2 + H'*d_h/2 + W'*d_w/2) bytes, rounded up to 256) plus,
  * unless flags has VA3D_K_ROTATED, the rotated keys (B*heads*N*head_dim*2
- * bytes).  Returns 0 for invalid arguments.  Host-only.
+ * bytes), plus scratch for splitting the query tiles of the last partial wave
+ * over two key halves (min(128, tiles) * 266,244 bytes, rounded up to 256,
+ * with tiles = B*heads*ceil(N/256)).  Returns 0 for invalid arguments.
+ * Host-only.
  */
 size_t va3d_workspace_bytes(int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
                             unsigned flags);
@@ -167,6 +171,39 @@ int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 
                         va3d_bf16 *o_spatial, va3d_bf16 *o_temporal, int B, int heads, int N,
                         int head_dim, const va3d_grid_t *grid, float softmax_scale,
                         unsigned flags, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of optional scratch attn_cross_fwd can use (for splitting the query
+ * tiles of the last partial wave over two key halves):
+ * min(128, B*heads*ceil(Nq/256)) * 266,244, rounded up to 256.  Returns 0
+ * for invalid arguments.  Host-only.
+ */
+size_t va3d_cross_workspace_bytes(int B, int heads, int Nq, int Nkv, int head_dim);
+
+/*
+ * Text cross-attention of a video block ("04 HunyuanVideo and Wan",
+ * note.shouss.top, section 3.1, the steps of one Wan block: queries from the
+ * video tokens, keys and values from the text encoder's tokens, up to 512 of
+ * them; the text side is not updated).  No RoPE on either side:
+ *   o = softmax(scale * q k^T) v,   lse = log-sum-exp of the row.
+ *   q     device, [B, heads, Nq, head_dim] bf16 (video tokens), read only.
+ *   k, v  device, [B, heads, Nkv, head_dim] bf16 (text tokens), read only;
+ *         any Nkv >= 1.
+ *   o     device, [B, heads, Nq, head_dim] bf16, written; must not overlap
+ *         the inputs or the workspace.
+ *   lse   device fp32 [B, heads, Nq] (natural log), or NULL.
+ *   softmax_scale  <= 0 selects 1/sqrt(head_dim).
+ *   workspace, workspace_bytes  optional device scratch, 256-byte aligned:
+ *         NULL (or too small) runs every tile whole; with
+ *         va3d_cross_workspace_bytes(...) bytes the last partial wave is
+ *         split.  Contents are overwritten.
+ * Accumulation is fp32; P is rounded to bf16 before the PV product; o is
+ * rounded to bf16 (nearest even).
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _ALIGNMENT, _DEVICE, _CUDA.
+ */
+int attn_cross_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *o,
+                   float *lse, int B, int heads, int Nq, int Nkv, int head_dim,
+                   float softmax_scale, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Capacity of the built-in scratch used by attn3d_full_fwd_noalloc. */
 #define VA3D_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)

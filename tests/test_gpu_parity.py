@@ -74,7 +74,7 @@ FACTORISED_SMALL = [si.WORKLOADS["tiny"], si.WORKLOADS["c17f480"], custom("f_odd
                     custom("f_t1", 1, 9, 15), custom("f_t33", 33, 2, 3), custom("f_t64", 64, 1, 5),
                     custom("f_hw1", 7, 1, 1), custom("f_b2", 4, 6, 7, batch=2)]
 
-LARGE = ["c81f480", "c81f720", "joint720"]
+LARGE = ["c81f480", "c81f720", "joint720", "refimg720"]
 
 
 # ------------------------------------------------------------------ RoPE
@@ -197,6 +197,44 @@ def test_factorised_single_pass_outputs(va):
     s2, t2 = va.attn_factorized_fwd(q, k, v, g)
     assert torch.equal(s_only.view(torch.int16), s2.view(torch.int16))
     assert torch.equal(t_only.view(torch.int16), t2.view(torch.int16))
+
+
+# ------------------------------------------------------- text cross-attention
+
+def cross_case(name, nq, nkv, heads=2, batch=1, seed=11):
+    # queries on a 1 x 1 x nq "grid" (the grid does not enter cross-attention)
+    return si.Workload(name, 1, 1, nq, heads, (44, 42, 42), batch=batch, seed=seed, n_kv=nkv)
+
+
+CROSS_SMALL = [cross_case("x_1_1", 1, 1, heads=1), cross_case("x_32_7", 32, 7),
+               cross_case("x_300_512", 300, 512, heads=3), cross_case("x_1000_129", 1000, 129, batch=2),
+               cross_case("x_257_1", 257, 1), cross_case("x_7800_512", 7800, 512, heads=12),
+               cross_case("x_130_1000", 130, 1000)]
+
+
+@pytest.mark.parametrize("w", CROSS_SMALL, ids=lambda w: w.name)
+def test_cross_attention_all_rows(va, w):
+    q, k, v = si.qkv(w)
+    o, lse = va.attn_cross_fwd(dev(q), dev(k), dev(v), return_lse=True)
+    ref, ref_lse = oracle.cross_attention(q, k, v, want_lse=True)
+    check(host(o).reshape(ref.shape), ref, f"cross {w.name}")
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(ref_lse.shape), ref_lse, atol=2e-3, rtol=0)
+    # without scratch every tile runs whole: same result within the bar
+    o2 = va.attn_cross_fwd(dev(q), dev(k), dev(v), workspace=torch.empty(0, dtype=torch.uint8,
+                                                                         device="cuda"))
+    check(host(o2).reshape(ref.shape), ref, f"cross {w.name} unsplit")
+    assert va.device_error() == 0
+
+
+def test_cross_attention_sampled_rows_full_size(va):
+    w = si.WORKLOADS["cross720"]
+    q, k, v = si.qkv(w)
+    rows = si.sample_rows(w, 512)
+    o = va.attn_cross_fwd(dev(q), dev(k), dev(v))
+    got = host(o[:, :, torch.from_numpy(rows).cuda(), :]).reshape(w.batch * w.heads, rows.size, 128)
+    ref = oracle.cross_attention(q, k, v, rows=rows)
+    check(got, ref, "cross cross720")
+    assert va.device_error() == 0
 
 
 def test_binding_rejects_bad_tensors(va):

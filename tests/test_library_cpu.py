@@ -30,9 +30,9 @@ def header_functions():
 
 def test_header_declares_the_boundary():
     names = header_functions()
-    for must in ("rope3d_apply", "attn3d_full_fwd", "attn_factorized_fwd",
-                 "va3d_grid_from_video", "va3d_workspace_bytes", "va3d_status_string",
-                 "va3d_device_error", "va3d_version"):
+    for must in ("rope3d_apply", "attn3d_full_fwd", "attn_factorized_fwd", "attn_cross_fwd",
+                 "va3d_grid_from_video", "va3d_workspace_bytes", "va3d_cross_workspace_bytes",
+                 "va3d_status_string", "va3d_device_error", "va3d_version"):
         assert must in names
 
 
@@ -87,6 +87,14 @@ def test_workspace_bytes(va):
     assert va.workspace_bytes(1, 12, 32760, bad) == 0
 
 
+def test_cross_workspace_bytes(va):
+    per = 2 * 256 * 128 * 4 + 2 * 256 * 8 + 4
+    assert va.cross_workspace_bytes(1, 40, 75600, 512) == (128 * per + 255) // 256 * 256
+    assert va.cross_workspace_bytes(2, 2, 1000, 129) == (16 * per + 255) // 256 * 256
+    assert va.cross_workspace_bytes(1, 2, 32, 0) == 0
+    assert va.lib.va3d_cross_workspace_bytes(1, 2, 32, 8, 64) == 0
+
+
 def test_status_strings(va):
     for code in range(0, -7, -1):
         assert va.lib.va3d_status_string(code)
@@ -119,6 +127,13 @@ def test_bad_arguments_rejected_before_any_device_call(va):
     gl = va.Grid.make(65, 1, 1)
     assert lib.attn_factorized_fwd(p, p, p, None, p, 1, 1, 65, 128, ctypes.byref(gl), 0.0, 0, p,
                                    1 << 20, None) == -2
+    # cross-attention: no keys, head_dim, misaligned output or workspace
+    assert lib.attn_cross_fwd(p, p, p, p, None, 1, 2, 32, 0, 128, 0.0, None, 0, None) == -1
+    assert lib.attn_cross_fwd(p, p, p, p, None, 1, 2, 32, 8, 64, 0.0, None, 0, None) == -2
+    assert lib.attn_cross_fwd(p, p, p, q, None, 1, 2, 32, 8, 128, 0.0, None, 0, None) == -3
+    assert lib.attn_cross_fwd(p, p, p, p, None, 1, 2, 32, 8, 128, 0.0,
+                              ctypes.c_void_p(p.value + 16), 4096, None) in (-3,)
+    assert lib.attn_cross_fwd(None, p, p, p, None, 1, 2, 32, 8, 128, 0.0, None, 0, None) == -1
     # odd RoPE range
     godd = va.Grid.make(2, 4, 4, dims=(43, 43, 42))
     assert lib.rope3d_apply(p, p, 1, 2, 32, 128, ctypes.byref(godd), None) == -1
@@ -134,6 +149,8 @@ def test_binding_has_no_cpu_path(va):
         va.rope3d_apply(x, g)
     with pytest.raises(ValueError, match="CUDA"):
         va.attn_factorized_fwd(x, x, x, g)
+    with pytest.raises(ValueError, match="CUDA"):
+        va.attn_cross_fwd(x, x, x)
 
 
 def test_product_and_oracle_share_nothing():
