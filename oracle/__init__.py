@@ -14,7 +14,9 @@ Two layers:
   factorised or full"), ``rope_3d_dims`` (section "Position: RoPE in three
   dimensions");
 * the fp64 C oracle (``va3d_oracle.c``) for RoPE and attention, reached with
-  ctypes: ``rope3d`` and ``attention``.
+  ctypes: ``rope3d``, ``attention`` (full, spatial, temporal, joint),
+  ``window_attention`` (local 3D windows) and ``cross_attention`` (video
+  queries over text keys).
 """
 from __future__ import annotations
 
@@ -160,6 +162,13 @@ def _load():
                                             ctypes.POINTER(ctypes.c_int),
                                             ctypes.POINTER(ctypes.c_int)]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_window_attention.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_long, ctypes.c_long, ctypes.c_int,
+                                                ctypes.POINTER(_Grid), ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                                                ctypes.c_void_p, ctypes.c_long, ctypes.c_void_p,
+                                                ctypes.c_void_p]
+        lib.oracle_window_attention.restype = ctypes.c_int
         lib.oracle_cross_attention.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                ctypes.c_long, ctypes.c_long, ctypes.c_long,
                                                ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
@@ -225,6 +234,32 @@ def attention(q_bits, k_bits, v_bits, grid: Grid, mode="full", rows=None, scale=
                                   lse.ctypes.data if want_lse else None)
     if rc != 0:
         raise ValueError(f"oracle_attention rejected the arguments ({rc})")
+    return (out, lse) if want_lse else out
+
+
+def window_attention(q_bits, k_bits, v_bits, grid: Grid, window, rows=None, scale=None,
+                     rotate=True, want_lse=False):
+    """fp64 local 3D-window attention (anthology record sota-390, the W.A.L.T
+    comparison): the grid is cut into non-overlapping windows of
+    ``window = (wt, wh, ww)`` tokens and every token attends to its own window,
+    3D RoPE as in full attention.  Returns out [BH, len(rows), d] (and lse)."""
+    q, k, v = _bits(q_bits), _bits(k_bits), _bits(v_bits)
+    N, D = q.shape[-2], q.shape[-1]
+    BH = int(np.prod(q.shape[:-2])) if q.ndim > 2 else 1
+    if rows is None:
+        rows = np.arange(N, dtype=np.int64)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.empty((BH, rows.size, D), dtype=np.float64)
+    lse = np.empty((BH, rows.size), dtype=np.float64) if want_lse else None
+    g = grid._c()
+    wt, wh, ww = (int(x) for x in window)
+    rc = _load().oracle_window_attention(q.ctypes.data, k.ctypes.data, v.ctypes.data, BH, N, D,
+                                         ctypes.byref(g), wt, wh, ww,
+                                         float(scale) if scale else 0.0, 1 if rotate else 0,
+                                         rows.ctypes.data, rows.size, out.ctypes.data,
+                                         lse.ctypes.data if want_lse else None)
+    if rc != 0:
+        raise ValueError(f"oracle_window_attention rejected the arguments ({rc})")
     return (out, lse) if want_lse else out
 
 

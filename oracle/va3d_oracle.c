@@ -17,6 +17,8 @@
  *    sequence-parallel shard listing).
  *  - "CogVideoX Architecture ..." (aifetchly-blog), section 3 "3D Rotary
  *    Position Embeddings": block-diagonal R_3D(t, y, x) and d_h = d_t+d_y+d_x.
+ *  - anthology-of-the-sota record sota-390 (CogVideoX's full-vs-factorised
+ *    comparison): W.A.L.T's blocks that attend inside local 3D windows.
  *  - "How AI Generates Video" (latentailabs), "What is 3D RoPE": Wan2.1 splits
  *    128 dims into 22/21/21 rotary pairs (axes_dim = [44, 42, 42]).
  *  - "04 HunyuanVideo and Wan" (note.shouss.top), section 2.5: head dim 128,
@@ -53,7 +55,7 @@ typedef struct {
     int off_t, off_h, off_w; /* coordinate offsets (0 for the method itself) */
 } oracle_grid;
 
-enum { ORACLE_FULL = 0, ORACLE_SPATIAL = 1, ORACLE_TEMPORAL = 2 };
+enum { ORACLE_FULL = 0, ORACLE_SPATIAL = 1, ORACLE_TEMPORAL = 2, ORACLE_WINDOW = 3 };
 
 enum {
     ORACLE_OK = 0,
@@ -159,7 +161,7 @@ int oracle_rope3d(const uint16_t *x, double *y, long BH, long N, int head_dim,
  * too); the spatial pass takes the H'W' tokens of i's frame; the temporal pass
  * takes the T' tokens at i's spatial position (h, w), one per frame.
  * Writes the key indices to keys[] and returns their count. */
-static long key_set(const oracle_grid *g, int mode, long i, long N, long *keys)
+static long key_set(const oracle_grid *g, int mode, const int *win, long i, long N, long *keys)
 {
     long cnt = 0;
     if (mode == ORACLE_FULL) {
@@ -171,8 +173,16 @@ static long key_set(const oracle_grid *g, int mode, long i, long N, long *keys)
     const long hw = (long)g->H * g->W;
     if (mode == ORACLE_SPATIAL) {
         for (long j = 0; j < hw; ++j) keys[cnt++] = (long)t * hw + j;
-    } else {
+    } else if (mode == ORACLE_TEMPORAL) {
         for (long tt = 0; tt < g->T; ++tt) keys[cnt++] = tt * hw + (long)h * g->W + w;
+    } else {
+        /* the tokens of the query's window: coordinates in
+         * [t0, t0 + wt) x [h0, h0 + wh) x [w0, w0 + ww), t0 = (t / wt) * wt, ... */
+        const int t0 = t / win[0] * win[0], h0 = h / win[1] * win[1], w0 = w / win[2] * win[2];
+        for (int tt = t0; tt < t0 + win[0]; ++tt)
+            for (int hh = h0; hh < h0 + win[1]; ++hh)
+                for (int ww = w0; ww < w0 + win[2]; ++ww)
+                    keys[cnt++] = tt * hw + (long)hh * g->W + ww;
     }
     return cnt;
 }
@@ -186,14 +196,15 @@ static long key_set(const oracle_grid *g, int mode, long i, long N, long *keys)
  * rows: nrows query indices in [0, N), the same for every bh.
  * out: fp64 [BH, nrows, head_dim]; lse: fp64 [BH, nrows] or NULL.
  */
-int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                     long BH, long N, int head_dim, const oracle_grid *g,
-                     int mode, double scale, int rotate, const long *rows,
-                     long nrows, double *out, double *lse)
+static int attention_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          long BH, long N, int head_dim, const oracle_grid *g,
+                          int mode, const int *win, double scale, int rotate, const long *rows,
+                          long nrows, double *out, double *lse)
 {
     if (!grid_ok(g, head_dim) || N != (long)g->T * g->H * g->W + g->n_text)
         return ORACLE_EINVAL;
-    if (mode != ORACLE_FULL && mode != ORACLE_SPATIAL && mode != ORACLE_TEMPORAL)
+    if (mode != ORACLE_FULL && mode != ORACLE_SPATIAL && mode != ORACLE_TEMPORAL &&
+        mode != ORACLE_WINDOW)
         return ORACLE_EINVAL;
     if (mode != ORACLE_FULL && g->n_text != 0) return ORACLE_EINVAL;
     for (long r = 0; r < nrows; ++r)
@@ -247,7 +258,7 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                     rope_row(g, head_dim, qx, qr, i);
                 else
                     memcpy(qr, qx, sizeof(double) * D);
-                const long nk = key_set(g, mode, i, N, keys);
+                const long nk = key_set(g, mode, win, i, N, keys);
 
                 /* scores and their maximum over the keys */
                 double m = -INFINITY;
@@ -281,6 +292,35 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     free(kr);
     free(vd);
     return ORACLE_OK;
+}
+
+int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     long BH, long N, int head_dim, const oracle_grid *g,
+                     int mode, double scale, int rotate, const long *rows,
+                     long nrows, double *out, double *lse)
+{
+    if (mode == ORACLE_WINDOW) return ORACLE_EINVAL;
+    return attention_impl(q, k, v, BH, N, head_dim, g, mode, NULL, scale, rotate, rows, nrows,
+                          out, lse);
+}
+
+/*
+ * Local 3D-window attention (anthology record sota-390, the W.A.L.T
+ * comparison: blocks that attend inside local 3D windows).  The grid is cut
+ * into non-overlapping windows of wt x wh x ww tokens (each dimension must
+ * divide the grid's); a token attends to the tokens of its own window, with
+ * the same 3D RoPE (absolute coordinates) as full attention.  No text tokens.
+ */
+int oracle_window_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            long BH, long N, int head_dim, const oracle_grid *g,
+                            int wt, int wh, int ww, double scale, int rotate,
+                            const long *rows, long nrows, double *out, double *lse)
+{
+    if (g->n_text != 0 || wt < 1 || wh < 1 || ww < 1) return ORACLE_EINVAL;
+    if (g->T % wt != 0 || g->H % wh != 0 || g->W % ww != 0) return ORACLE_EINVAL;
+    const int win[3] = {wt, wh, ww};
+    return attention_impl(q, k, v, BH, N, head_dim, g, ORACLE_WINDOW, win, scale, rotate, rows,
+                          nrows, out, lse);
 }
 
 /*

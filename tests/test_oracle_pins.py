@@ -438,6 +438,78 @@ def test_oracle_rejects_bad_arguments():
 
 
 # ---------------------------------------------------------------------------
+# local 3D-window attention (W.A.L.T blocks, anthology record sota-390)
+# ---------------------------------------------------------------------------
+
+def _window_mask(grid, win):
+    t, h, w = _coords(grid)
+    wt, wh, ww = win
+    return ((t[:, None] // wt == t[None, :] // wt) & (h[:, None] // wh == h[None, :] // wh)
+            & (w[:, None] // ww == w[None, :] // ww))
+
+
+@pytest.mark.parametrize("win", [(2, 2, 3), (1, 4, 2), (4, 1, 6), (2, 4, 6)])
+def test_window_equals_masked_full(win):
+    """Window attention = full attention under the mask 'same window'."""
+    g = Grid(4, 4, 6)
+    q, k, v = (_rand_bits((2, g.N, 128), s) for s in (131, 132, 133))
+    o, lse = oracle.window_attention(q, k, v, g, win, want_lse=True)
+    qr, kr = oracle.rope3d(q, g), oracle.rope3d(k, g)
+    mask = _window_mask(g, win)
+    np.testing.assert_allclose(o, _sdpa(qr, kr, bf16_bits_to_f64(v), mask=mask), atol=1e-12, rtol=0)
+    s = torch.from_numpy(qr @ kr.transpose(0, 2, 1) / math.sqrt(128))
+    s = s.masked_fill(~torch.from_numpy(mask), -math.inf)
+    np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), atol=1e-12, rtol=0)
+
+
+def test_window_special_cases_reduce_to_the_other_modes():
+    g = Grid(3, 4, 5)
+    q, k, v = (_rand_bits((1, g.N, 128), s) for s in (134, 135, 136))
+    pairs = [((3, 4, 5), "full"), ((1, 4, 5), "spatial"), ((3, 1, 1), "temporal")]
+    for win, mode in pairs:
+        np.testing.assert_allclose(oracle.window_attention(q, k, v, g, win),
+                                   oracle.attention(q, k, v, g, mode=mode), atol=1e-13, rtol=0)
+    # one-token windows: every row copies its own value
+    o = oracle.window_attention(q, k, v, g, (1, 1, 1))
+    np.testing.assert_array_equal(o, bf16_bits_to_f64(v))
+    # windows are defined on grid coordinates, RoPE on relative ones: a shift
+    # of every position leaves the output unchanged
+    gs = Grid(3, 4, 5, offset=(5, 9, 2))
+    np.testing.assert_allclose(oracle.window_attention(q, k, v, gs, (3, 2, 5)),
+                               oracle.window_attention(q, k, v, g, (3, 2, 5)), atol=1e-9, rtol=0)
+
+
+def test_window_brute_force_tiny():
+    g = Grid(2, 4, 4)
+    q, k, v = (_rand_bits((1, g.N, 128), s) for s in (137, 138, 139))
+    win = (1, 2, 4)
+    o = oracle.window_attention(q, k, v, g, win)[0]
+    t, h, w = _coords(g)
+    Rs = [_explicit_R((t[i], h[i], w[i]), (44, 42, 42)) for i in range(g.N)]
+    qf, kf, vf = (bf16_bits_to_f64(x)[0] for x in (q, k, v))
+    qr = np.stack([Rs[i] @ qf[i] for i in range(g.N)])
+    kr = np.stack([Rs[i] @ kf[i] for i in range(g.N)])
+    for i in range(g.N):
+        keys = [j for j in range(g.N) if t[j] == t[i] and h[j] // 2 == h[i] // 2]
+        s_ = np.array([qr[i] @ kr[j] for j in keys]) / math.sqrt(128)
+        p_ = np.exp(s_ - s_.max())
+        np.testing.assert_allclose(o[i], (p_[:, None] * vf[keys]).sum(0) / p_.sum(), atol=2e-5,
+                                   rtol=0)
+
+
+def test_window_rejects_bad_arguments():
+    g = Grid(3, 4, 6)
+    x = np.zeros((1, g.N, 128), dtype=np.uint16)
+    for win in [(2, 2, 3), (1, 3, 3), (1, 4, 5), (0, 1, 1)]:
+        with pytest.raises(ValueError):
+            oracle.window_attention(x, x, x, g, win)
+    gt = Grid(3, 4, 6, n_text=2)
+    xt = np.zeros((1, gt.N, 128), dtype=np.uint16)
+    with pytest.raises(ValueError):
+        oracle.window_attention(xt, xt, xt, gt, (1, 2, 3))
+
+
+# ---------------------------------------------------------------------------
 # text cross-attention (Wan block, "04 HunyuanVideo and Wan" section 3.1)
 # ---------------------------------------------------------------------------
 
