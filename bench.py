@@ -445,6 +445,18 @@ def extras(va, device, stream, peak_tf, peak_gbs):
         "full_over_factorised_time": round(full_ms / (sp_ms + tp_ms), 2),
         "full_over_factorised_flops": round(f_full / (f_sp + 4.0 * HEAD_DIM * w.heads * hw * w.T ** 2), 2),
     }
+    # local 3D windows of 3 x 9 x 16 = 432 tokens on the same clip (keys pre-rotated)
+    win = (3, 9, 16)
+    vol = win[0] * win[1] * win[2]
+    _, w_ms = timed_loop(ev_pair(lambda: va.attn_window_fwd(q, kr, v, g, win, k_rotated=True,
+                                                              out=o, workspace=ws)), 10, 3, 1, device)
+    f_w = 4.0 * w.N * vol * HEAD_DIM * w.heads
+    t_f = f_w / (peak_tf * 1e12) * 1e3
+    t_b = tbytes / (peak_gbs * 1e9) * 1e3
+    out["window720"] = {"window": list(win), "tokens": w.N, "heads": w.heads, "ms": round(w_ms, 4),
+                        "tflops": round(f_w / w_ms / 1e9, 1), "gbs": round(tbytes / w_ms / 1e6, 1),
+                        "roofline_ms": round(max(t_f, t_b), 4),
+                        "frac_of_roofline": round(max(t_f, t_b) / w_ms, 4)}
     del q, k, v, kr, o, o2, ws
     torch.cuda.empty_cache()
 

@@ -12,6 +12,7 @@ Entry points (same names as the C ABI):
 * ``attn3d_full_fwd(q, k, v, grid)``        full 3D (or joint video+text) attention
 * ``attn_factorized_fwd(q, k, v, grid)``    spatial and temporal passes
 * ``attn_cross_fwd(q, k, v)``               video-to-text cross-attention (no RoPE)
+* ``attn_window_fwd(q, k, v, grid, window)`` local 3D-window attention
 * ``grid_from_video(frames, height, width)``  token grid of a clip
 * ``workspace_bytes(...)``, ``device_error()``
 """
@@ -30,7 +31,8 @@ HEAD_DIM = 128
 SYMBOLS = ("va3d_status_string", "va3d_version", "va3d_grid_from_video",
            "va3d_workspace_bytes", "rope3d_apply", "attn3d_full_fwd",
            "attn_factorized_fwd", "va3d_device_error", "attn3d_full_fwd_noalloc",
-           "va3d_cross_workspace_bytes", "attn_cross_fwd")
+           "va3d_cross_workspace_bytes", "attn_cross_fwd", "attn_window_fwd",
+           "va3d_watchdog_selftest")
 
 
 class VA3DError(RuntimeError):
@@ -81,10 +83,12 @@ def _load():
     lib.attn3d_full_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp, sz, vp]
     lib.attn_factorized_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp, sz, vp]
     lib.va3d_device_error.argtypes = [i]
+    lib.va3d_watchdog_selftest.argtypes = [vp]
     lib.attn3d_full_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, f, u, vp]
     lib.va3d_cross_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.va3d_cross_workspace_bytes.restype = sz
     lib.attn_cross_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+    lib.attn_window_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, i, i, i, f, u, vp, sz, vp]
     return lib
 
 
@@ -249,6 +253,35 @@ def attn_factorized_fwd(q, k, v, grid, *, spatial=True, temporal=True, scale=Non
     return out_spatial, out_temporal
 
 
+def attn_window_fwd(q, k, v, grid, window, *, scale=None, return_lse=False, k_rotated=False,
+                    out=None, lse=None, workspace=None):
+    """Local 3D-window attention: tokens attend inside non-overlapping windows
+    of ``window = (wt, wh, ww)`` tokens (each dividing the grid), 3D RoPE as in
+    full attention.  Returns o (and lse if asked)."""
+    torch = _torch()
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    B, H, N, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N)
+                            or not lse.is_contiguous() or not lse.is_cuda):
+        raise ValueError("lse must be a contiguous CUDA float32 [B, heads, N] tensor")
+    ws = _workspace(q, grid, k_rotated, workspace)
+    wt, wh, ww = (int(x) for x in window)
+    rc = lib.attn_window_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
+                             ctypes.byref(grid), wt, wh, ww, float(scale or 0.0),
+                             VA3D_K_ROTATED if k_rotated else 0, _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(q))
+    if rc != VA3D_OK:
+        raise VA3DError("attn_window_fwd", rc)
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
 def cross_workspace_bytes(B, heads, Nq, Nkv):
     return int(lib.va3d_cross_workspace_bytes(B, heads, Nq, Nkv, HEAD_DIM))
 
@@ -283,6 +316,14 @@ def attn_cross_fwd(q, k, v, *, scale=None, return_lse=False, out=None, lse=None,
     if rc != VA3D_OK:
         raise VA3DError("attn_cross_fwd", rc)
     return (out, lse) if (return_lse or lse is not None) else out
+
+
+def watchdog_selftest():
+    """Launch the watchdog probe on the current device (its wait times out by
+    design after 2 s); read the result with device_error()."""
+    rc = lib.va3d_watchdog_selftest(ctypes.c_void_p(_torch().cuda.current_stream().cuda_stream))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_watchdog_selftest", rc)
 
 
 def device_error(reset=True):

@@ -106,7 +106,29 @@ struct AttnArgs {
     __nv_bfloat16 *o;
     float *lse;        // may be null
     RopeParams rp;
+    // Local 3D windows (win != 0): segment s is window s of the grid in
+    // (t, h, w) raster order of windows, its rows the window's tokens in
+    // (dt, dh, dw) raster order.  Rows are gathered token by token from the
+    // natural-order tensors below (no TMA), and O and LSE rows are written
+    // back to the tokens' natural positions.
+    int win;
+    int win_t, win_h, win_w;   // window size
+    int nwin_h, nwin_w;        // windows along h and w
+    const __nv_bfloat16 *gq, *gk, *gv;
 };
+
+// Natural token index of row `local` of window `seg`.
+__device__ __forceinline__ int window_token(const AttnArgs &a, int seg, int local) {
+    const int dw = local % a.win_w;
+    const int rest = local / a.win_w;
+    const int dh = rest % a.win_h;
+    const int dt = rest / a.win_h;
+    const int cw = seg % a.nwin_w;
+    const int rest2 = seg / a.nwin_w;
+    const int ch = rest2 % a.nwin_h;
+    const int ct = rest2 / a.nwin_h;
+    return ((ct * a.win_t + dt) * a.rp.H + ch * a.win_h + dh) * a.rp.W + cw * a.win_w + dw;
+}
 
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
     // K-major, 128 B swizzle: 8-row groups 1024 B apart; the leading offset
@@ -184,10 +206,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(bar(B_QFULL), 1);
         mbar_init(bar(B_QREADY0), BM);
         mbar_init(bar(B_QREADY1), BM);
+        // full barriers: one TMA arrival with its byte count, or one arrival
+        // per gathering thread in window mode
+        const uint32_t full_count = a.win ? 64u : 1u;
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar(B_KFULL0 + s), 1);
+            mbar_init(bar(B_KFULL0 + s), full_count);
             mbar_init(bar(B_KEMPTY0 + s), 1);
-            mbar_init(bar(B_VFULL0 + s), 1);
+            mbar_init(bar(B_VFULL0 + s), full_count);
             mbar_init(bar(B_VEMPTY0 + s), 1);
         }
         mbar_init(bar(B_SFULL0), 1);
@@ -212,10 +237,83 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (warp >= 8) {
     regs_lower<kProducerRegs>();
     if (warp >= 10) {
-        // idle
+        // ------------------------------------------- gathering loader (windows)
+        // 64 threads copy the K and V rows of each key tile token by token
+        // (16-byte cp.async into the same swizzled layout TMA produces), two
+        // tiles in flight; after its copies land a thread fences them for the
+        // tensor core's proxy and arrives on the tile's full barrier.
+        if (a.win) {
+            const int lt = threadIdx.x - 10 * 32;   // 0..63
+            auto gather = [&](const __nv_bfloat16 *src, uint32_t dst, int j) {
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int i = lt * 2 + h2;                 // row of the tile
+                    const int local = (j0 + j) * BN + i;       // row of the window
+                    const uint32_t row = dst + i * 128;
+                    if (local < a.kv_len) {
+                        const __nv_bfloat16 *g =
+                            src + (static_cast<size_t>(bh) * a.N + window_token(a, seg, local)) * HD;
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            cp_async16(row + (c >> 3) * kHalfBytes + (((c & 7) ^ (i & 7)) << 4), g + c * 8);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            st_shared_zero16(row + (c >> 3) * kHalfBytes + (((c & 7) ^ (i & 7)) << 4));
+                    }
+                }
+            };
+            // Commit groups go K(0), V(0), K(1), V(1), ...  Step j publishes
+            // K(j-1) and V(j-1) as soon as each has landed and issues K(j) and
+            // V(j) once their stages are released, so up to one K and one V
+            // tile are in flight besides the ones being published.
+            bool ok = true;
+            for (int j = 0; j <= n_kv && ok; ++j) {
+                const int s = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                if (j >= 1) {
+                    cp_async_wait<1>();                  // K(j-1); V(j-1) may be pending
+                    fence_proxy_async_smem();
+                    mbar_arrive(bar(B_KFULL0 + ((j - 1) & 1)));
+                }
+                if (j < n_kv) {
+                    if (j >= kStages &&
+                        !(ok = mbar_wait(bar(B_KEMPTY0 + s), ph ^ 1, abort_flag, VA3D_DEVERR_TIMEOUT_LOAD)))
+                        break;
+                    gather(a.gk, sbase + OFF_K + s * kTileBytes, j);
+                    cp_async_commit();
+                }
+                if (j >= 1) {
+                    if (j < n_kv)
+                        cp_async_wait<1>();              // V(j-1); K(j) may be pending
+                    else
+                        cp_async_wait<0>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(bar(B_VFULL0 + ((j - 1) & 1)));
+                }
+                if (j < n_kv) {
+                    if (j >= kStages &&
+                        !(ok = mbar_wait(bar(B_VEMPTY0 + s), ph ^ 1, abort_flag, VA3D_DEVERR_TIMEOUT_LOAD)))
+                        break;
+                    gather(a.gv, sbase + OFF_V + s * kTileBytes, j);
+                    cp_async_commit();
+                }
+            }
+            cp_async_wait<0>();
+            if (ok) {
+                // every released stage was consumed; wait for the last tiles'
+                // releases so no arrival lands after the CTA exits
+                const int first = n_kv > kStages ? n_kv - kStages : 0;
+                for (int j = first; j < n_kv && ok; ++j)
+                    ok = mbar_wait(bar(B_KEMPTY0 + (j & 1)), (j >> 1) & 1, abort_flag,
+                                   VA3D_DEVERR_TIMEOUT_LOAD) &&
+                         mbar_wait(bar(B_VEMPTY0 + (j & 1)), (j >> 1) & 1, abort_flag,
+                                   VA3D_DEVERR_TIMEOUT_LOAD);
+            }
+        }
     } else if (warp == 9) {
         // ------------------------------------------------------------ loader
-        if (lane == 0) {
+        if (lane == 0 && !a.win) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
@@ -352,12 +450,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint32_t taO = tmem + lane_addr + (g ? COL_O1 : COL_O0);
         const int n = q0 + g * BM + r;            // token index of this row
 
-        bool ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QFULL), 0, abort_flag,
-                                                    VA3D_DEVERR_TIMEOUT_SOFTMAX));
-        if (ok) {
-            if (a.rope_q) rope_q_row(smem + OFF_Q + g * kTileBytes, r, n, a);
+        // natural token index of this row (differs from n only for windows)
+        const int n_out = a.win && n < seg_end ? window_token(a, seg, n - seg_start) : n;
+        bool ok = true;
+        if (a.win) {
+            // gather this row of Q itself (256 contiguous bytes) into the
+            // swizzled tile; rows past the window are zero
+            uint8_t *tile = smem + OFF_Q + g * kTileBytes;
+            const bool in = n < seg_end;
+            uint4 row[16];
+            if (in) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    a.gq + (static_cast<size_t>(bh) * a.N + n_out) * HD);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) row[c] = __ldg(src + c);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                *reinterpret_cast<uint4 *>(tile + (c >> 3) * kHalfBytes + r * 128 +
+                                           (((c & 7) ^ (r & 7)) << 4)) = row[c];
+            if (a.rope_q && in) rope_q_row(tile, r, n_out, a);
             fence_proxy_async_smem();
             mbar_arrive(bar(g ? B_QREADY1 : B_QREADY0));
+        } else {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QFULL), 0, abort_flag,
+                                                   VA3D_DEVERR_TIMEOUT_SOFTMAX));
+            if (ok) {
+                if (a.rope_q) rope_q_row(smem + OFF_Q + g * kTileBytes, r, n, a);
+                fence_proxy_async_smem();
+                mbar_arrive(bar(g ? B_QREADY1 : B_QREADY0));
+            }
         }
 
         float m_ref = -INFINITY;   // running row maximum, log2 units (scaled)
@@ -458,7 +583,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tc_fence_after();
             const float inv_l = 1.0f / l;
             const bool valid = n < seg_end;
-            uint4 *dst = reinterpret_cast<uint4 *>(a.o + (static_cast<size_t>(bh) * a.N + n) * HD);
+            uint4 *dst = reinterpret_cast<uint4 *>(a.o + (static_cast<size_t>(bh) * a.N + n_out) * HD);
             if (!split) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -479,7 +604,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     }
                 }
                 if (a.lse != nullptr && valid)
-                    a.lse[static_cast<size_t>(bh) * a.N + n] = (m_ref + log2f(l)) * 0.69314718055994531f;
+                    a.lse[static_cast<size_t>(bh) * a.N + n_out] = (m_ref + log2f(l)) * 0.69314718055994531f;
             } else {
                 // half of the keys: store the normalised partial and its (max, sum)
                 const size_t prow = (static_cast<size_t>(split_idx) * 2 + part) * (2 * BM) + g * BM + r;
@@ -533,7 +658,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                                                 pack_bf16x2(x1.z * c_s + y1.z * c_o, x1.w * c_s + y1.w * c_o));
                     }
                     if (a.lse != nullptr && valid)
-                        a.lse[static_cast<size_t>(bh) * a.N + n] =
+                        a.lse[static_cast<size_t>(bh) * a.N + n_out] =
                             (m_max + log2f(w_s + w_o)) * 0.69314718055994531f;
                 }
             }

@@ -17,6 +17,7 @@
 #include "rope.cuh"
 #include "attn_sm100.cuh"
 #include "attn_temporal.cuh"
+#include "selftest.cuh"
 
 using namespace va3d;
 
@@ -188,9 +189,12 @@ SplitScratch split_scratch(void *base, size_t bytes) {
 // Q is [BH, N, 128] in n_seg segments of seg_len rows; K and V are
 // [BH, Nkv, 128] in n_seg segments of kv_len rows; segment s of the queries
 // attends to segment s of the keys.
+// win (optional): local 3D window size; segments are then the windows, their
+// rows gathered token by token (seg_len == kv_len == window volume).
 int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float *lse, int BH, int N,
                 int Nkv, int seg_len, int kv_len, int n_seg, bool rope_q, const RopeParams &rp,
-                const float2 *tab, float scale, const SplitScratch &sc, cudaStream_t st) {
+                const float2 *tab, float scale, const SplitScratch &sc, cudaStream_t st,
+                const int *win = nullptr) {
     CUtensorMap mq, mk, mv;
     int rc;
     if ((rc = make_map(&mq, q, N, BH, fa::BM)) != VA3D_OK) return rc;
@@ -208,6 +212,17 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
     a.o = static_cast<__nv_bfloat16 *>(o);
     a.lse = lse;
     a.rp = rp;
+    if (win != nullptr) {
+        a.win = 1;
+        a.win_t = win[0];
+        a.win_h = win[1];
+        a.win_w = win[2];
+        a.nwin_h = rp.H / win[1];
+        a.nwin_w = rp.W / win[2];
+        a.gq = static_cast<const __nv_bfloat16 *>(q);
+        a.gk = static_cast<const __nv_bfloat16 *>(k_rot);
+        a.gv = static_cast<const __nv_bfloat16 *>(v);
+    }
     a.n_seg = n_seg;
     // One CTA per SM.  If the last wave of tiles would fill at most half of the
     // SMs and every tile has at least two 128-key steps, each of its tiles is
@@ -456,6 +471,33 @@ int attn_cross_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, v
     if ((rc = launch_table(nullptr, sc.count, sc.capacity, none, st)) != VA3D_OK) return rc;
     return launch_attn(q, k, v, o, lse, B * heads, Nq, Nkv, Nq, Nkv, 1, false, none, nullptr, scale,
                        sc, st);
+}
+
+int attn_window_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *o,
+                    float *lse, int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
+                    int win_t, int win_h, int win_w, float softmax_scale, unsigned flags,
+                    void *workspace, size_t workspace_bytes, void *stream) {
+    if (o == nullptr || grid == nullptr) return VA3D_ERR_INVALID;
+    if (!aligned16(o) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return VA3D_ERR_ALIGNMENT;
+    if (grid->n_text != 0 || win_t < 1 || win_h < 1 || win_w < 1) return VA3D_ERR_INVALID;
+    if (grid->T % win_t != 0 || grid->H % win_h != 0 || grid->W % win_w != 0) return VA3D_ERR_INVALID;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Prepared p;
+    int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
+                     workspace_bytes, true, st, &p);
+    if (rc != VA3D_OK) return rc;
+    const int win[3] = {win_t, win_h, win_w};
+    const int vol = win_t * win_h * win_w;
+    return launch_attn(q, p.k_rot, v, o, lse, B * heads, N, N, vol, vol, N / vol, true, p.rp, p.tab,
+                       p.scale, p.split, st, win);
+}
+
+int va3d_watchdog_selftest(void *stream) {
+    int rc;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    watchdog_probe_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>();
+    return launch_status();
 }
 
 int va3d_device_error(int reset) {

@@ -17,7 +17,10 @@
  *  - joint video+text attention: "04 HunyuanVideo and Wan" (note.shouss.top)
  *    sections 2.3-2.4, and the handbook's diffusers example (video tokens +
  *    text tokens attended together in one sequence);
- *  - text cross-attention: the same page, section 3.1 (Wan's block).
+ *  - text cross-attention: the same page, section 3.1 (Wan's block);
+ *  - local 3D-window attention: anthology-of-the-sota record sota-390
+ *    (W.A.L.T's local 3D-window blocks, the one numbered comparison against
+ *    full attention it cites).
  *
  * Conventions shared by every entry point
  *  - Tensors are contiguous bf16 (bit patterns, va3d_bf16) of shape
@@ -84,7 +87,8 @@ enum {
     VA3D_DEVERR_NONE = 0,
     VA3D_DEVERR_TIMEOUT_LOAD = 1,     /* a wait in the tile-loading role timed out */
     VA3D_DEVERR_TIMEOUT_MMA = 2,      /* a wait in the MMA-issuing role timed out */
-    VA3D_DEVERR_TIMEOUT_SOFTMAX = 3   /* a wait in the softmax role timed out */
+    VA3D_DEVERR_TIMEOUT_SOFTMAX = 3,  /* a wait in the softmax role timed out */
+    VA3D_DEVERR_TIMEOUT_SELFTEST = 4  /* the wait of va3d_watchdog_selftest timed out (expected) */
 };
 
 /* Human-readable text of a status code; never NULL. */
@@ -173,6 +177,24 @@ int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 
                         unsigned flags, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Local 3D-window attention (anthology-of-the-sota record sota-390, the
+ * W.A.L.T comparison: blocks whose tokens attend only inside local 3D
+ * windows).  The grid is cut into non-overlapping windows of
+ * win_t x win_h x win_w tokens (each must divide T', H', W'); every video
+ * token attends to the tokens of its own window, with the same 3D RoPE
+ * (absolute coordinates) as full attention:
+ *   o_i = softmax_j(scale * RoPE(q_i) . RoPE(k_j)) v_j over j in window(i).
+ * grid->n_text must be 0.  win = (T', H', W') is full attention, (1, H', W')
+ * the spatial pass, (T', 1, 1) the temporal pass.  Other arguments, the
+ * workspace size (va3d_workspace_bytes with the same grid and flags),
+ * results and errors as in attn3d_full_fwd.
+ */
+int attn_window_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *o,
+                    float *lse, int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
+                    int win_t, int win_h, int win_w, float softmax_scale, unsigned flags,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of optional scratch attn_cross_fwd can use (for splitting the query
  * tiles of the last partial wave over two key halves):
  * min(128, B*heads*ceil(Nq/256)) * 266,244, rounded up to 256.  Returns 0
@@ -236,6 +258,17 @@ int attn3d_full_fwd_noalloc(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_b
                             va3d_bf16 *o, float *lse, int B, int heads, int N, int head_dim,
                             const va3d_grid_t *grid, float softmax_scale, unsigned flags,
                             void *stream);
+
+/*
+ * Watchdog self-test: launches one CTA whose mbarrier wait can never
+ * complete (the arrival it waits for is never made).  The bounded wait gives
+ * up after its limit (2 s), records VA3D_DEVERR_TIMEOUT_SELFTEST in the
+ * device error word (unless another code is already there) and the kernel
+ * exits; no trap, no fault, the context stays usable.  Asynchronous on
+ * `stream`; read the result with va3d_device_error().
+ * Errors: VA3D_ERR_DEVICE, _CUDA.
+ */
+int va3d_watchdog_selftest(void *stream);
 
 /*
  * Last device-side watchdog code recorded on the current device

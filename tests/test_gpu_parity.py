@@ -76,6 +76,9 @@ FACTORISED_SMALL = [si.WORKLOADS["tiny"], si.WORKLOADS["c17f480"], custom("f_odd
 
 LARGE = ["c81f480", "c81f720", "joint720", "refimg720"]
 
+# the local window timed on the 720p clip: 3 x 9 x 16 = 432 tokens
+WINDOW_720 = (3, 9, 16)
+
 
 # ------------------------------------------------------------------ RoPE
 
@@ -197,6 +200,123 @@ def test_factorised_single_pass_outputs(va):
     s2, t2 = va.attn_factorized_fwd(q, k, v, g)
     assert torch.equal(s_only.view(torch.int16), s2.view(torch.int16))
     assert torch.equal(t_only.view(torch.int16), t2.view(torch.int16))
+
+
+# ------------------------------------------------------ local 3D windows
+
+WINDOW_SMALL = [(si.WORKLOADS["tiny"], (1, 2, 4)), (si.WORKLOADS["tiny"], (2, 2, 2)),
+                (si.WORKLOADS["tiny"], (1, 1, 1)), (si.WORKLOADS["c17f480"], (5, 6, 4)),
+                (si.WORKLOADS["c17f480"], (1, 10, 26)), (si.WORKLOADS["c17f480"], (5, 15, 13)),
+                (custom("w_odd", 3, 5, 17, heads=3), (3, 5, 1)),
+                (custom("w_b2", 2, 7, 9, batch=2), (2, 7, 3))]
+
+
+def window_keys(w, win, n):
+    """Token indices of the window that holds token n."""
+    hw = w.H * w.W
+    t, rem = divmod(int(n), hw)
+    h, x = divmod(rem, w.W)
+    t0, h0, x0 = t // win[0] * win[0], h // win[1] * win[1], x // win[2] * win[2]
+    return np.array([(tt * w.H + hh) * w.W + xx for tt in range(t0, t0 + win[0])
+                     for hh in range(h0, h0 + win[1]) for xx in range(x0, x0 + win[2])])
+
+
+def window_bounds(w, win, q, k, v, rows, want_o=True):
+    """Per-element bound on |GPU - oracle| for window attention, derived from
+    the kernel's arithmetic to first order.  The scores use Q~ and K~ rounded
+    to bf16, so |ds_j| <= D_j = 2^-8 * scale * sum_i |q~_i| |k~_ji|; a score
+    error moves o_c by sum_j p_j ds_j (v_jc - o_c) and the LSE by
+    sum_j p_j ds_j.  P rounded to bf16 adds 2^-9 sum_j p_j |v_jc|, the
+    polynomial exp2 (relative error 7.5e-5) 1.5e-4 sum_j p_j |v_jc - o_c|, the
+    bf16 output 2^-9 |o_c|.  Returns (bound_o [BH, rows, 128] or None,
+    bound_lse [BH, rows]).  Worst case over the rounding errors, so several
+    times the typical error."""
+    g = ogrid(w)
+    scale = 1.0 / np.sqrt(128)
+    BH = w.batch * w.heads
+    qb, kb, vb = (x.reshape(BH, w.N, 128) for x in (q, k, v))
+    bo = np.empty((BH, rows.size, 128)) if want_o else None
+    bl = np.empty((BH, rows.size))
+    # group the rows by window: rows of one window share its keys
+    groups = {}
+    for i, n in enumerate(rows):
+        ks = window_keys(w, win, n)
+        groups.setdefault(int(ks[0]), (ks, []))[1].append(i)
+    for b in range(BH):
+        qr = oracle.rope3d(qb[b:b + 1], g)[0]
+        kr = oracle.rope3d(kb[b:b + 1], g)[0]
+        vf = bf16_bits_to_f64(vb[b])
+        for ks, idx in groups.values():
+            idx = np.array(idx)
+            qs = qr[rows[idx]]                              # [r, 128]
+            sc = qs @ kr[ks].T * scale                       # [r, keys]
+            p = np.exp(sc - sc.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            o = p @ vf[ks]                                   # [r, 128]
+            D = 2.0 ** -8 * scale * (np.abs(qs) @ np.abs(kr[ks]).T)     # [r, keys]
+            pd = p * D
+            bl[b, idx] = pd.sum(axis=1) * 1.1 + 2e-4
+            if want_o:
+                dv = np.abs(vf[ks][None, :, :] - o[:, None, :])         # [r, keys, 128]
+                bo[b, idx] = (np.einsum("rk,rkc->rc", pd, dv)
+                              + 1.5e-4 * np.einsum("rk,rkc->rc", p, dv)
+                              + 2.0 ** -9 * (p @ np.abs(vf[ks])) + 2.0 ** -9 * np.abs(o)) * 1.1 + 1e-6
+    return bo, bl
+
+
+def check_window(got, ref, bound, label):
+    """Within the derived per-element bound, and the mean-abs and relative-L2
+    bars of the other modes."""
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), f"{label}: non-finite output"
+    worst = float((err / bound).max())
+    assert worst <= 1.0, f"{label}: error reaches {worst:.2f} x the derived bound"
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    assert float(err.mean()) <= MEAN_ABS and rel <= REL_L2, (label, float(err.mean()), rel)
+    return float(err.max()), worst
+
+
+@pytest.mark.parametrize("w,win", WINDOW_SMALL, ids=lambda x: x.name if hasattr(x, "name") else
+                         "x".join(map(str, x)))
+def test_window_attention_all_rows(va, w, win):
+    q, k, v = si.qkv(w)
+    o, lse = va.attn_window_fwd(dev(q), dev(k), dev(v), vgrid(va, w), win, return_lse=True)
+    ref, ref_lse = oracle.window_attention(q, k, v, ogrid(w), win, want_lse=True)
+    # outputs: the bar of the other modes; LSE: the derived bound (with a
+    # handful of keys per window there is no averaging of score errors)
+    check(host(o).reshape(ref.shape), ref, f"window {w.name} {win}")
+    _, bl = window_bounds(w, win, q, k, v, np.arange(w.N), want_o=False)
+    lerr = np.abs(lse.cpu().numpy().reshape(ref_lse.shape) - ref_lse)
+    assert (lerr <= bl).all(), float((lerr / bl).max())
+    assert va.device_error() == 0
+
+
+def test_window_gather_matches_the_tma_paths_bit_for_bit(va):
+    """A window of the whole grid is full attention and a window of one frame
+    the spatial pass: the gathered rows are then in natural order, so the
+    outputs must equal the TMA-loaded paths bit for bit."""
+    w = si.WORKLOADS["c17f480"]
+    q, k, v = (dev(x) for x in si.qkv(w))
+    g = vgrid(va, w)
+    full = va.attn3d_full_fwd(q, k, v, g)
+    win_full = va.attn_window_fwd(q, k, v, g, (w.T, w.H, w.W))
+    assert torch.equal(full.view(torch.int16), win_full.view(torch.int16))
+    sp, _ = va.attn_factorized_fwd(q, k, v, g, temporal=False)
+    win_sp = va.attn_window_fwd(q, k, v, g, (1, w.H, w.W))
+    assert torch.equal(sp.view(torch.int16), win_sp.view(torch.int16))
+
+
+def test_window_attention_sampled_rows_full_size(va):
+    w = si.WORKLOADS["c81f720"]
+    win = WINDOW_720
+    q, k, v = si.qkv(w)
+    rows = si.sample_rows(w, 512)
+    o = va.attn_window_fwd(dev(q), dev(k), dev(v), vgrid(va, w), win)
+    got = host(o[:, :, torch.from_numpy(rows).cuda(), :]).reshape(w.batch * w.heads, rows.size, 128)
+    ref = oracle.window_attention(q, k, v, ogrid(w), win, rows=rows)
+    bo, _ = window_bounds(w, win, q, k, v, rows)
+    check_window(got, ref, bo, f"window c81f720 {win}")
+    assert va.device_error() == 0
 
 
 # ------------------------------------------------------- text cross-attention

@@ -31,6 +31,7 @@ def header_functions():
 def test_header_declares_the_boundary():
     names = header_functions()
     for must in ("rope3d_apply", "attn3d_full_fwd", "attn_factorized_fwd", "attn_cross_fwd",
+                 "attn_window_fwd", "va3d_watchdog_selftest",
                  "va3d_grid_from_video", "va3d_workspace_bytes", "va3d_cross_workspace_bytes",
                  "va3d_status_string", "va3d_device_error", "va3d_version"):
         assert must in names
@@ -134,6 +135,17 @@ def test_bad_arguments_rejected_before_any_device_call(va):
     assert lib.attn_cross_fwd(p, p, p, p, None, 1, 2, 32, 8, 128, 0.0,
                               ctypes.c_void_p(p.value + 16), 4096, None) in (-3,)
     assert lib.attn_cross_fwd(None, p, p, p, None, 1, 2, 32, 8, 128, 0.0, None, 0, None) == -1
+    # window attention: window must divide the grid; no text tokens
+    gw = va.Grid.make(2, 4, 4)
+    assert lib.attn_window_fwd(p, p, p, p, None, 1, 2, 32, 128, ctypes.byref(gw), 1, 3, 4, 0.0, 0,
+                               p, 1 << 20, None) == -1
+    assert lib.attn_window_fwd(p, p, p, p, None, 1, 2, 32, 128, ctypes.byref(gw), 0, 2, 4, 0.0, 0,
+                               p, 1 << 20, None) == -1
+    gwt = va.Grid.make(2, 4, 4, n_text=2)
+    assert lib.attn_window_fwd(p, p, p, p, None, 1, 2, 34, 128, ctypes.byref(gwt), 1, 2, 4, 0.0, 0,
+                               p, 1 << 20, None) == -1
+    assert lib.attn_window_fwd(p, p, p, p, None, 1, 2, 32, 64, ctypes.byref(gw), 1, 2, 4, 0.0, 0,
+                               p, 1 << 20, None) == -2
     # odd RoPE range
     godd = va.Grid.make(2, 4, 4, dims=(43, 43, 42))
     assert lib.rope3d_apply(p, p, 1, 2, 32, 128, ctypes.byref(godd), None) == -1
@@ -151,6 +163,8 @@ def test_binding_has_no_cpu_path(va):
         va.attn_factorized_fwd(x, x, x, g)
     with pytest.raises(ValueError, match="CUDA"):
         va.attn_cross_fwd(x, x, x)
+    with pytest.raises(ValueError, match="CUDA"):
+        va.attn_window_fwd(x, x, x, g, (1, 2, 2))
 
 
 def test_product_and_oracle_share_nothing():
