@@ -103,6 +103,12 @@ struct Cfg {
 // Shared memory per warp: (Q, K, V) with T rows of 256 bytes.
 __host__ __device__ inline int temporal_warp_bytes(int T) { return 3 * T * 256; }
 
+// Shared memory for the block's copy of the angle table's t section
+// (T * d_t/2 (cos, sin) pairs), rounded up to 16 bytes.
+__host__ __device__ inline int temporal_table_bytes(int T, int half_t) {
+    return (T * half_t * 8 + 15) / 16 * 16;
+}
+
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
@@ -157,10 +163,12 @@ template <bool kRotate>
 __device__ __forceinline__ int rotate_to_f16(uint8_t *tile, const __nv_bfloat16 *src, size_t base,
                                              size_t tstride, int T, int rlane, int cch,
                                              const float2 (&cs_fixed)[4], const bool (&is_t)[4],
-                                             const TemporalArgs &a, bool rotate) {
+                                             const float2 *t_tab, bool rotate) {
+    // t pairs: the block's shared copy of the t section (entry j*T + t);
+    // h and w pairs: fixed for the task
     auto angle = [&](int r, int e) -> float2 {
         if (!rotate) return make_float2(1.f, 0.f);
-        return is_t[e] ? a.rope_tab[r * a.rp.half_t + cch * 4 + e] : cs_fixed[e];
+        return is_t[e] ? t_tab[(cch * 4 + e) * T + r] : cs_fixed[e];
     };
     float mx = 0.f;
     for (int r = rlane; r < T; r += 2) {
@@ -201,9 +209,18 @@ temporal_kernel(const __grid_constant__ TemporalArgs a) {
     const long long total = static_cast<long long>(a.BH) * a.HW;
     const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
     long long task = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + warp;
-    if (task >= total) return;   // the whole warp leaves together; no block barrier is used
 
-    uint8_t *sq = smem + warp * temporal_warp_bytes(T);   // Q (raw, fp16 rotated, then bf16 O)
+    // The t angles vary per row of every task: the block keeps a copy of the
+    // table's t section in shared memory (read-only after this barrier, the
+    // only block-wide barrier).
+    float2 *t_tab = reinterpret_cast<float2 *>(smem);
+    const int n_t = T * a.rp.half_t;
+    for (int i = threadIdx.x; i < n_t; i += blockDim.x) t_tab[i] = a.rope_tab[i];
+    __syncthreads();
+    if (task >= total) return;   // the whole warp leaves together
+
+    uint8_t *sq = smem + temporal_table_bytes(T, a.rp.half_t) + warp * temporal_warp_bytes(T);
+    // sq: Q (raw, fp16 rotated, then bf16 O)
     uint8_t *sk = sq + tensor_bytes;                     // K (raw, then fp16 rotated)
     uint8_t *sv = sk + tensor_bytes;                     // V (bf16)
     const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv);
@@ -245,8 +262,9 @@ temporal_kernel(const __grid_constant__ TemporalArgs a) {
         }
         cp_async_wait<0>();
         __syncwarp();
-        const int eq = rotate_to_f16<true>(sq, a.q, base, tstride, T, rlane, cch, cs_fixed, is_t, a, true);
-        const int ek = rotate_to_f16<true>(sk, a.k, base, tstride, T, rlane, cch, cs_fixed, is_t, a,
+        const int eq = rotate_to_f16<true>(sq, a.q, base, tstride, T, rlane, cch, cs_fixed, is_t, t_tab,
+                                           true);
+        const int ek = rotate_to_f16<true>(sk, a.k, base, tstride, T, rlane, cch, cs_fixed, is_t, t_tab,
                                            a.rope_k != 0);
         const float scale_log2 = a.scale_log2 * pow2f(-(eq + ek));
         __syncwarp();

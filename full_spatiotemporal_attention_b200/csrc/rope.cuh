@@ -21,6 +21,7 @@ struct RopeParams {
     int pe_t, pe_h;            // pairs [0,pe_t) turn with t, [pe_t,pe_h) with h, the rest with w
     int half_t, half_h, half_w;  // pairs per axis (d_axis / 2)
     int tab_h, tab_w;          // table offsets (entries) of the h and w sections; t is at 0
+                               // (each section pair-major: entry (j, pos) at j * extent + pos)
     int tab_entries;           // T*half_t + H*half_h + W*half_w
     float inv_freq[64];        // per pair; computed on the host in fp64, rounded to fp32
 };
@@ -37,11 +38,13 @@ __device__ __forceinline__ float2 rope_cs(float inv_freq, int pos) {
     return make_float2(c, s);
 }
 
-// Table entry of pair p at axis position pos (same layout as rope_table_kernel).
+// Table entry of pair p for a token at (t, h, w) (same layout as
+// rope_table_kernel).  Pair-major sections: threads that hold consecutive
+// tokens (consecutive w) read consecutive entries for the same pair.
 __device__ __forceinline__ int table_index(const RopeParams &rp, int p, int t, int h, int w) {
-    if (p < rp.pe_t) return t * rp.half_t + p;
-    if (p < rp.pe_h) return rp.tab_h + h * rp.half_h + (p - rp.pe_t);
-    return rp.tab_w + w * rp.half_w + (p - rp.pe_h);
+    if (p < rp.pe_t) return p * rp.T + t;
+    if (p < rp.pe_h) return rp.tab_h + (p - rp.pe_t) * rp.H + h;
+    return rp.tab_w + (p - rp.pe_h) * rp.W + w;
 }
 
 // (x0, x1) -> (x0 c - x1 s, x0 s + x1 c) on one packed bf16 pair.
@@ -52,8 +55,8 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t packed, float2 cs) {
     return pack_bf16x2(y0, y1);
 }
 
-// Build the cos/sin table for a grid: entries (t, j) at t*half_t + j, then
-// (h, j) at tab_h + h*half_h + j, then (w, j) at tab_w + w*half_w + j.
+// Build the cos/sin table for a grid: entries (j, t) at j*T + t, then
+// (j, h) at tab_h + j*H + h, then (j, w) at tab_w + j*W + w.
 // It also clears `n_zero` ints at `zero` (per-call counters of the attention
 // kernel that follows on the same stream).
 __global__ void rope_table_kernel(float2 *__restrict__ tab, int *__restrict__ zero, int n_zero,
@@ -64,16 +67,18 @@ __global__ void rope_table_kernel(float2 *__restrict__ tab, int *__restrict__ ze
          e += gridDim.x * blockDim.x) {
         int p, pos;
         if (e < rp.tab_h) {
-            pos = e / rp.half_t;
-            p = e - pos * rp.half_t;
+            p = e / rp.T;
+            pos = e - p * rp.T;
         } else if (e < rp.tab_w) {
-            int r = e - rp.tab_h;
-            pos = r / rp.half_h;
-            p = rp.pe_t + (r - pos * rp.half_h);
+            const int r = e - rp.tab_h;
+            const int j = r / rp.H;
+            pos = r - j * rp.H;
+            p = rp.pe_t + j;
         } else {
-            int r = e - rp.tab_w;
-            pos = r / rp.half_w;
-            p = rp.pe_h + (r - pos * rp.half_w);
+            const int r = e - rp.tab_w;
+            const int j = r / rp.W;
+            pos = r - j * rp.W;
+            p = rp.pe_h + j;
         }
         tab[e] = rope_cs(rp.inv_freq[p], pos);
     }

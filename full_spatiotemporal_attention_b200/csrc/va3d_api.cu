@@ -259,9 +259,10 @@ int launch_temporal_t(const tp::TemporalArgs &a, cudaStream_t st) {
     // grid is persistent (at most the resident blocks), each warp strides
     // over (batch*head, position) tasks.
     const int warp_bytes = tp::temporal_warp_bytes(a.T);
-    const int budget = tp::Cfg<MAXT>::kSmemBudget;
+    const int table_bytes = tp::temporal_table_bytes(a.T, a.rp.half_t);
+    const int budget = tp::Cfg<MAXT>::kSmemBudget - table_bytes;
     const int warps = std::max(1, std::min(tp::Cfg<MAXT>::kMaxWarps, budget / warp_bytes));
-    const int smem = warps * warp_bytes;
+    const int smem = table_bytes + warps * warp_bytes;
     const int per_sm = std::max(1, std::min(4, (216 * 1024) / smem));
     if (cudaFuncSetAttribute(tp::temporal_kernel<MAXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
