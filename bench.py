@@ -45,6 +45,9 @@ def parse_args():
     p.add_argument("--no-extras", action="store_true", help="skip the secondary measurements")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
+    p.add_argument("--case", choices=["temporal720", "spatial720", "window720", "cross720"],
+                   help="run only this secondary kernel (warm-up + --steps launches, one "
+                        "JSON line); a small, single-kernel command for profilers")
     return p.parse_args()
 
 
@@ -504,6 +507,49 @@ def extras(va, device, stream, peak_tf, peak_gbs):
     return out
 
 
+def run_case(args):
+    """One secondary kernel alone on the 720p clip (keys pre-rotated), for
+    profiling: `--warmup` untimed and `--steps` timed launches."""
+    import torch
+    import full_spatiotemporal_attention_b200 as va
+    import seeded_inputs as si
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w = si.WORKLOADS["cross720" if args.case == "cross720" else "c81f720"]
+    q, k, v = (to_dev(x, device) for x in si.qkv(w))
+    o = torch.empty_like(q)
+    if args.case == "cross720":
+        ws = torch.empty(va.cross_workspace_bytes(w.batch, w.heads, w.N, w.n_kv), dtype=torch.uint8,
+                         device=device)
+        fn = lambda: va.attn_cross_fwd(q, k, v, out=o, workspace=ws)
+    else:
+        g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+        kr = va.rope3d_apply(k, g)
+        ws = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g, k_rotated=True),
+                         dtype=torch.uint8, device=device)
+        if args.case == "temporal720":
+            fn = lambda: va.attn_factorized_fwd(q, kr, v, g, spatial=False, k_rotated=True,
+                                                out_temporal=o, workspace=ws)
+        elif args.case == "spatial720":
+            fn = lambda: va.attn_factorized_fwd(q, kr, v, g, temporal=False, k_rotated=True,
+                                                out_spatial=o, workspace=ws)
+        else:
+            fn = lambda: va.attn_window_fwd(q, kr, v, g, (3, 9, 16), k_rotated=True, out=o,
+                                            workspace=ws)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        return a, b
+    _, ms = timed_loop(step, args.steps, args.warmup, 1, device)
+    return {"case": args.case, "workload": w.description, "ms": round(ms, 4),
+            "device_error": va.device_error()}
+
+
 def bench_reference(args, rank, world):
     """The oracle, as it stands, on the host cores: each step computes a
     bounded sample of query rows of the same workload."""
@@ -546,6 +592,9 @@ def main():
         world = int(os.environ.get("WORLD_SIZE", "1"))
         if rank == 0:
             print(json.dumps(bench_reference(args, rank, world)), flush=True)
+        return
+    if args.case:
+        print(json.dumps(run_case(args)), flush=True)
         return
     rank, world, local = init_dist("nccl")
     line = bench_ours(args, rank, world, local)
