@@ -7,26 +7,36 @@
 // full 3D attention and joint video+text attention use one segment of N
 // tokens (handbook "How attention sees time": every token together); the
 // spatial pass of factorised attention uses T' segments of H'W' tokens (one
-// per frame).  The score matrix is never materialised (online softmax).
+// per frame); local 3D windows use one segment per window, rows gathered token
+// by token; text cross-attention ("04 HunyuanVideo and Wan", section 3.1) uses
+// one segment of video queries over a separate key/value tensor (the text
+// tokens), with no rotation.  The score matrix is never materialised (online
+// softmax).
 //
-// CTA = one (batch*head, segment, 256 query rows) work tile, one CTA per SM:
-//   warps 0-3   softmax group 0: rows of query tile 0 (thread = TMEM lane = row)
-//   warps 4-7   softmax group 1: rows of query tile 1
-//   warp  8     tcgen05.mma issuer (one thread) and TMEM allocator
-//   warp  9     TMA loader (one thread)
-//   warps 10-11 idle (they complete the producer warpgroup for setmaxnreg)
+// CTA = one (batch*head, segment, NQ x 128 query rows) work tile (KCfg):
+//   NQ = 2 (one CTA per SM)      NQ = 1 (two CTAs per SM, short key loops)
+//   warps 0-3  softmax group 0   warps 0-3  softmax group 0
+//   warps 4-7  softmax group 1   warp  4    MMA issuer, TMEM owner
+//   warp  8    MMA issuer        warp  5    TMA loader
+//   warp  9    TMA loader        warps 6-7  gathering loaders (windows)
+//   warps 10-11 gathering loaders (windows)
+// A softmax thread owns one query row (= TMEM lane).
 //
-// Work units (1-D grid): units below n_whole each cover one 256-row tile over
-// all keys of its segment.  When the last wave would leave SMs idle, its tiles
+// Work units (1-D grid): units below n_whole each cover one NQ x 128-row tile
+// over all keys of its segment.  When the last wave would leave SMs idle, its tiles
 // are instead covered by two units each, one per half of the key tiles; each
 // half writes its normalised fp32 output with its row maximum and sum to the
 // workspace, and the second half to finish (a per-tile counter) merges the
 // two and writes O.
-// TMEM (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1, 128 columns each;
-// P (bf16 pairs) overwrites the first 64 columns of its S.  The MMA issuer
-// ping-pongs the two query tiles so that one tile's softmax overlaps the
-// other tile's QK^T and PV products.  Q, K, V tiles are 128 rows x 128 bf16,
-// loaded by TMA as two 64-column boxes with the 128-byte swizzle.
+//
+// TMEM (256 NQ columns x 128 lanes, fp32): S_g at 128 g, O_g at 128 (NQ + g);
+// P (bf16 pairs) overwrites the first 64 columns of its S.  With NQ = 2 the
+// MMA issuer ping-pongs the two query tiles so that one tile's softmax
+// overlaps the other tile's QK^T and PV products; with NQ = 1 the two CTAs of
+// an SM interleave on its tensor core in the same way, and one CTA's
+// prologue and epilogue overlap the other's main loop.  Q, K, V tiles are
+// 128 rows x 128 bf16, loaded by TMA as two 64-column boxes with the 128-byte
+// swizzle.
 #pragma once
 
 #include <type_traits>
@@ -40,22 +50,8 @@ namespace fa {
 constexpr int BM = 128;                    // query rows per tile
 constexpr int BN = 128;                    // keys per tile
 constexpr int HD = 128;                    // head dim
-constexpr int kStages = 2;                 // K and V ring depth
-constexpr int kThreads = 384;             // three warpgroups
-// Register split after launch (168 per thread at launch = 64,512 per block):
-// the two softmax warpgroups take 216, the producer warpgroup keeps 72;
-// 2 * 128 * 216 + 128 * 72 = 64,512.
-constexpr int kSoftmaxRegs = 216;
-constexpr int kProducerRegs = 72;
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * 168,
-              "register split exceeds the launch allocation");
 constexpr int kTileBytes = BM * HD * 2;    // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2; // one 64-column box: 128 rows x 128 B
-
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + 2 * kTileBytes;
-constexpr int OFF_V = OFF_K + kStages * kTileBytes;
-constexpr int OFF_BAR = OFF_V + kStages * kTileBytes;
 
 enum Bar {
     B_QFULL = 0,
@@ -73,14 +69,37 @@ enum Bar {
     NUM_BARS
 };
 
-constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
-constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
-constexpr int OFF_MERGE = OFF_ABORT + 8;     // int: this unit merges the two halves
-constexpr int kSmemUsed = OFF_MERGE + 8;
-constexpr int kSmemBytes = kSmemUsed + 1024;   // slack to align the base to 1024 B
-
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 384;
+// Configuration by NQ, the query tiles a CTA holds:
+//  NQ = 2: two softmax warpgroups ping-pong on one tensor core, a 2-stage
+//          K/V ring, one CTA per SM (long key sequences);
+//  NQ = 1: one softmax warpgroup and one K/V stage per CTA, two CTAs per SM
+//          that interleave on the tensor core, so that one CTA's prologue and
+//          epilogue overlap the other's main loop (short key sequences).
+// Warps 0 .. 4NQ-1 are the softmax groups; warp 4NQ issues MMAs and owns
+// TMEM, warp 4NQ+1 loads tiles, warps 4NQ+2 and 4NQ+3 gather (windows).
+template <int NQ>
+struct KCfg {
+    static constexpr int kStages = NQ == 2 ? 2 : 1;          // K and V ring depth
+    static constexpr int kThreads = 128 * (NQ + 1);
+    static constexpr int kMinBlocks = NQ == 2 ? 1 : 2;       // CTAs per SM
+    static constexpr int kLaunchRegs = NQ == 2 ? 168 : 128;  // per thread at launch
+    // setmaxnreg split (multiples of 8): NQ * 128 * softmax + 128 * producer
+    // must fit kThreads * kLaunchRegs.
+    static constexpr int kSoftmaxRegs = NQ == 2 ? 216 : 208;
+    static constexpr int kProducerRegs = NQ == 2 ? 72 : 48;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + NQ * kTileBytes;
+    static constexpr int OFF_V = OFF_K + kStages * kTileBytes;
+    static constexpr int OFF_BAR = OFF_V + kStages * kTileBytes;
+    static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
+    static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
+    static constexpr int OFF_MERGE = OFF_ABORT + 8;   // int: this unit merges the two halves
+    static constexpr int kSmemBytes = OFF_MERGE + 8 + 1024;   // slack to align the base
+    static constexpr uint32_t kTmemCols = 256 * NQ;   // S_g at 128 g, O_g at 128 (NQ + g)
+    static constexpr int kProdWarp = 4 * NQ;
+    static_assert(NQ * 128 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs,
+                  "register split exceeds the launch allocation");
+};
 
 // Lazy rescaling: a row keeps its running maximum (log2 units) until a new
 // score exceeds it by more than this; P values then stay below 2^8.
@@ -172,14 +191,24 @@ __device__ __forceinline__ void rope_q_row(uint8_t *tile, int r, int n, const At
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int NQ>
+__global__ void __launch_bounds__(KCfg<NQ>::kThreads, KCfg<NQ>::kMinBlocks)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
+    using C = KCfg<NQ>;
+    constexpr int kStages = C::kStages;
+    constexpr int OFF_Q = C::OFF_Q, OFF_K = C::OFF_K, OFF_V = C::OFF_V;
+    constexpr int OFF_TMEM_SLOT = C::OFF_TMEM_SLOT, OFF_MERGE = C::OFF_MERGE;
+    constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 128 * NQ, COL_O1 = 128 * NQ + 128;
+    constexpr int kMma = C::kProdWarp, kLoad = C::kProdWarp + 1, kGather = C::kProdWarp + 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const uint32_t sbase = smem_u32(smem);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
-    auto bar = [&](int i) -> uint32_t { return sbase + OFF_BAR + 8 * i; };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
+    auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
+    // tile j of the K/V stream: stage and phase of the ring
+    auto stg = [](int j) { return j % kStages; };
+    auto phs = [](int j) -> uint32_t { return static_cast<uint32_t>((j / kStages) & 1); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -194,7 +223,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int bh = tile / (a.q_blocks * a.n_seg);
     const int seg_start = seg * a.seg_len;
     const int seg_end = seg_start + a.seg_len;
-    const int q0 = seg_start + qb * (2 * BM);
+    const int q0 = seg_start + qb * (NQ * BM);
     const int kv_start = seg * a.kv_len;
     const int n_kv_all = (a.kv_len + BN - 1) / BN;
     const int kv_last_valid = a.kv_len - (n_kv_all - 1) * BN;
@@ -221,29 +250,29 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(bar(B_PFULL1), BM);
         mbar_init(bar(B_OFULL), 1);
         mbar_init(bar(B_DRAIN), 1);
-        mbar_init(bar(B_EPI), 2 * BM);
+        mbar_init(bar(B_EPI), NQ * BM);
         mbar_init(bar(B_EPI_GO), 1);
         *abort_flag = 0;
         mbar_init_fence();
         fence_proxy_async_smem();
     }
-    if (warp == 8) tmem_alloc(sbase + OFF_TMEM_SLOT, kTmemCols);
+    if (warp == kMma) tmem_alloc(sbase + OFF_TMEM_SLOT, C::kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_TMEM_SLOT);
     // Each role runs inside the branch that set its register budget (the new
     // budget applies to the code that instruction dominates).
-    if (warp >= 8) {
-    regs_lower<kProducerRegs>();
-    if (warp >= 10) {
+    if (warp >= kMma) {
+    regs_lower<C::kProducerRegs>();
+    if (warp >= kGather) {
         // ------------------------------------------- gathering loader (windows)
         // 64 threads copy the K and V rows of each key tile token by token
         // (16-byte cp.async into the same swizzled layout TMA produces), two
         // tiles in flight; after its copies land a thread fences them for the
         // tensor core's proxy and arrives on the tile's full barrier.
         if (a.win) {
-            const int lt = threadIdx.x - 10 * 32;   // 0..63
+            const int lt = threadIdx.x - kGather * 32;   // 0..63
             auto gather = [&](const __nv_bfloat16 *src, uint32_t dst, int j) {
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
@@ -269,12 +298,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             // tile are in flight besides the ones being published.
             bool ok = true;
             for (int j = 0; j <= n_kv && ok; ++j) {
-                const int s = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
+                const int s = stg(j);
+                const uint32_t ph = phs(j);
                 if (j >= 1) {
                     cp_async_wait<1>();                  // K(j-1); V(j-1) may be pending
                     fence_proxy_async_smem();
-                    mbar_arrive(bar(B_KFULL0 + ((j - 1) & 1)));
+                    mbar_arrive(bar(B_KFULL0 + stg(j - 1)));
                 }
                 if (j < n_kv) {
                     if (j >= kStages &&
@@ -289,7 +318,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     else
                         cp_async_wait<0>();
                     fence_proxy_async_smem();
-                    mbar_arrive(bar(B_VFULL0 + ((j - 1) & 1)));
+                    mbar_arrive(bar(B_VFULL0 + stg(j - 1)));
                 }
                 if (j < n_kv) {
                     if (j >= kStages &&
@@ -305,30 +334,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 // releases so no arrival lands after the CTA exits
                 const int first = n_kv > kStages ? n_kv - kStages : 0;
                 for (int j = first; j < n_kv && ok; ++j)
-                    ok = mbar_wait(bar(B_KEMPTY0 + (j & 1)), (j >> 1) & 1, abort_flag,
+                    ok = mbar_wait(bar(B_KEMPTY0 + stg(j)), phs(j), abort_flag,
                                    VA3D_DEVERR_TIMEOUT_LOAD) &&
-                         mbar_wait(bar(B_VEMPTY0 + (j & 1)), (j >> 1) & 1, abort_flag,
+                         mbar_wait(bar(B_VEMPTY0 + stg(j)), phs(j), abort_flag,
                                    VA3D_DEVERR_TIMEOUT_LOAD);
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == kLoad) {
         // ------------------------------------------------------------ loader
         if (lane == 0 && !a.win) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(bar(B_QFULL), 2 * kTileBytes);
-            for (int i = 0; i < 2; ++i)
+            mbar_arrive_expect_tx(bar(B_QFULL), NQ * kTileBytes);
+            for (int i = 0; i < NQ; ++i)
                 for (int hf = 0; hf < 2; ++hf)
                     tma_load_3d(sbase + OFF_Q + i * kTileBytes + hf * kHalfBytes, &tmQ,
                                 bar(B_QFULL), hf * 64, q0 + i * BM, bh);
-            // Tile j goes to stage j & 1 with phase (j >> 1) & 1; only the last
+            // Tile j goes to stage stg(j) with phase phs(j); only the last
             // kStages issued tiles can still be in flight or unreleased.
             int k_issued = 0, v_issued = 0;
             bool ok = true;
             for (int j = 0; j < n_kv; ++j) {
-                const int s = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
+                const int s = stg(j);
+                const uint32_t ph = phs(j);
                 const int kv0 = kv_start + (j0 + j) * BN;
                 if (j >= kStages &&
                     !(ok = mbar_wait(bar(B_KEMPTY0 + s), ph ^ 1, abort_flag, VA3D_DEVERR_TIMEOUT_LOAD)))
@@ -353,22 +382,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 // Producer tail: wait until the last tile of each stage has been
                 // released, so no barrier arrival can land after the CTA exits.
                 for (int j = k_first; j < k_issued && ok; ++j)
-                    ok = mbar_wait(bar(B_KEMPTY0 + (j & 1)), (j >> 1) & 1, abort_flag,
+                    ok = mbar_wait(bar(B_KEMPTY0 + stg(j)), phs(j), abort_flag,
                                    VA3D_DEVERR_TIMEOUT_LOAD);
                 for (int j = v_first; j < v_issued && ok; ++j)
-                    ok = mbar_wait(bar(B_VEMPTY0 + (j & 1)), (j >> 1) & 1, abort_flag,
+                    ok = mbar_wait(bar(B_VEMPTY0 + stg(j)), phs(j), abort_flag,
                                    VA3D_DEVERR_TIMEOUT_LOAD);
             }
             if (!ok) {
                 // Let the copies already in flight land before the CTA exits.
                 mbar_wait_drain(bar(B_QFULL), 0);
                 for (int j = k_first; j < k_issued; ++j)
-                    mbar_wait_drain(bar(B_KFULL0 + (j & 1)), (j >> 1) & 1);
+                    mbar_wait_drain(bar(B_KFULL0 + stg(j)), phs(j));
                 for (int j = v_first; j < v_issued; ++j)
-                    mbar_wait_drain(bar(B_VFULL0 + (j & 1)), (j >> 1) & 1);
+                    mbar_wait_drain(bar(B_VFULL0 + stg(j)), phs(j));
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == kMma) {
         // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, 0);
@@ -392,27 +421,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             };
 
             bool ok = mbar_wait(bar(B_QREADY0), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA) &&
-                      mbar_wait(bar(B_QREADY1), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA) &&
+                      (NQ == 1 || mbar_wait(bar(B_QREADY1), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA)) &&
                       mbar_wait(bar(B_KFULL0), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
             if (ok) {
                 tc_fence_after();
                 issue_s(0, 0);
                 mma_commit(bar(B_SFULL0));
-                issue_s(1, 0);
-                mma_commit(bar(B_SFULL1));
+                if constexpr (NQ == 2) {
+                    issue_s(1, 0);
+                    mma_commit(bar(B_SFULL1));
+                }
                 mma_commit(bar(B_KEMPTY0));
             }
             for (int j = 0; j < n_kv && ok; ++j) {
-                const int s = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
+                const int s = stg(j);
+                const uint32_t ph = phs(j);
                 const bool more = j + 1 < n_kv;
-                const int s2 = (j + 1) & 1;
-                const uint32_t ph2 = ((j + 1) >> 1) & 1;
+                const int s2 = stg(j + 1);
+                const uint32_t ph2 = phs(j + 1);
                 ok = mbar_wait(bar(B_VFULL0 + s), ph, abort_flag, VA3D_DEVERR_TIMEOUT_MMA) &&
                      mbar_wait(bar(B_PFULL0), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
                 if (!ok) break;
                 tc_fence_after();
                 issue_pv(0, s, j > 0);
+                // one query tile: V's stage is free after this product.  (Its
+                // release must not wait for the next QK^T: with one stage the
+                // gathering loader publishes that K tile only after refilling V.)
+                if constexpr (NQ == 1) mma_commit(bar(B_VEMPTY0 + s));
                 if (more) {
                     ok = mbar_wait(bar(B_KFULL0 + s2), ph2, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
                     if (!ok) break;
@@ -420,14 +455,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     issue_s(0, s2);
                     mma_commit(bar(B_SFULL0));
                 }
-                ok = mbar_wait(bar(B_PFULL1), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
-                if (!ok) break;
-                tc_fence_after();
-                issue_pv(1, s, j > 0);
-                mma_commit(bar(B_VEMPTY0 + s));
+                if constexpr (NQ == 2) {
+                    ok = mbar_wait(bar(B_PFULL1), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(1, s, j > 0);
+                    mma_commit(bar(B_VEMPTY0 + s));
+                }
                 if (more) {
-                    issue_s(1, s2);
-                    mma_commit(bar(B_SFULL1));
+                    if constexpr (NQ == 2) {
+                        issue_s(1, s2);
+                        mma_commit(bar(B_SFULL1));
+                    }
                     mma_commit(bar(B_KEMPTY0 + s2));
                 }
             }
@@ -441,7 +480,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
     }
     } else {
-        regs_raise<kSoftmaxRegs>();
+        regs_raise<C::kSoftmaxRegs>();
         // ---------------------------------------------------------- softmax
         const int g = warp >> 2;                  // query tile of this group
         const int r = ((warp & 3) << 5) + lane;   // row in the tile = TMEM lane
@@ -608,6 +647,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             } else {
                 // half of the keys: store the normalised partial and its (max, sum)
                 const size_t prow = (static_cast<size_t>(split_idx) * 2 + part) * (2 * BM) + g * BM + r;
+                // (the scratch holds 256 rows per half whatever NQ)
                 float4 *po = reinterpret_cast<float4 *>(a.part_o + prow * HD);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -668,7 +708,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 8) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kMma) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 }  // namespace fa

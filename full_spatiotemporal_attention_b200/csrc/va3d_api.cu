@@ -76,6 +76,13 @@ size_t tensor_bytes(int B, int heads, int N) {
 // normalised fp32 partial outputs of 256 rows, their (max, sum) and a counter.
 // At most kMaxSplit tiles are split (half of the SMs of a GPU with up to 256).
 constexpr int kMaxSplit = 128;
+// Segments of at most this many 128-key tiles (e.g. text cross-attention over
+// up to 512 text tokens) run one query tile per CTA, two CTAs per SM: there
+// the per-CTA prologue and epilogue weigh most and overlapping them across
+// CTAs pays (+10 % at 4 key tiles).  Longer segments keep two tiles per CTA
+// (one CTA per SM is 10-15 % faster from 29 key tiles on), and so do windows,
+// whose gathered K/V rows would be fetched twice as often.
+constexpr int kOneTileMaxKeyTiles = 4;
 constexpr size_t kSplitOBytes = 2 * 256 * 128 * 4;
 constexpr size_t kSplitMLBytes = 2 * 256 * 8;
 
@@ -205,7 +212,11 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
     a.N = N;
     a.seg_len = seg_len;
     a.kv_len = kv_len;
-    a.q_blocks = (seg_len + 2 * fa::BM - 1) / (2 * fa::BM);
+    // two query tiles per CTA for long key sequences; one (two CTAs per SM)
+    // when a unit's key loop is short and its prologue and epilogue weigh
+    const int n_kv_tiles = (kv_len + fa::BN - 1) / fa::BN;
+    const int nq = win == nullptr && n_kv_tiles <= kOneTileMaxKeyTiles ? 1 : 2;
+    a.q_blocks = (seg_len + nq * fa::BM - 1) / (nq * fa::BM);
     a.scale_log2 = static_cast<float>(scale * kLog2e);
     a.rope_q = rope_q ? 1 : 0;
     a.rope_tab = tab;
@@ -232,20 +243,33 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return VA3D_ERR_CUDA;
     const long long tiles = static_cast<long long>(BH) * n_seg * a.q_blocks;
-    const long long tail = sms > 0 ? tiles % sms : 0;
+    const long long resident = static_cast<long long>(sms) * (nq == 2 ? fa::KCfg<2>::kMinBlocks
+                                                                      : fa::KCfg<1>::kMinBlocks);
+    const long long tail = resident > 0 ? tiles % resident : 0;
     const int n_kv = (kv_len + fa::BN - 1) / fa::BN;
     long long split = 0;
-    if (tail > 0 && 2 * tail <= sms && tail <= sc.capacity && n_kv >= 2) split = tail;
+    if (tail > 0 && 2 * tail <= resident && tail <= sc.capacity && n_kv >= 2) split = tail;
     a.n_whole = static_cast<int>(tiles - split);
     a.part_o = sc.part_o;
     a.part_ml = sc.part_ml;
     a.part_count = sc.count;
-    if (cudaFuncSetAttribute(fa::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fa::kSmemBytes) != cudaSuccess)
-        return VA3D_ERR_CUDA;
     const long long units = tiles + split;
     if (units > 0x7fffffffll) return VA3D_ERR_UNSUPPORTED;
-    fa::attn_fwd_kernel<<<static_cast<unsigned>(units), fa::kThreads, fa::kSmemBytes, st>>>(mq, mk, mv, a);
+    if (nq == 2) {
+        using C = fa::KCfg<2>;
+        if (cudaFuncSetAttribute(fa::attn_fwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes) != cudaSuccess)
+            return VA3D_ERR_CUDA;
+        fa::attn_fwd_kernel<2><<<static_cast<unsigned>(units), C::kThreads, C::kSmemBytes, st>>>(
+            mq, mk, mv, a);
+    } else {
+        using C = fa::KCfg<1>;
+        if (cudaFuncSetAttribute(fa::attn_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes) != cudaSuccess)
+            return VA3D_ERR_CUDA;
+        fa::attn_fwd_kernel<1><<<static_cast<unsigned>(units), C::kThreads, C::kSmemBytes, st>>>(
+            mq, mk, mv, a);
+    }
     return launch_status();
 }
 
