@@ -12,12 +12,18 @@
 //  - only the T' real rows are staged; m16n8k16 fragments that reach past
 //    row T'-1 read row T'-1 again (their scores are masked or their outputs
 //    dropped), so nothing is zero-filled;
-//  - Q and K are turned by 3D RoPE in shared memory from the angle table and
-//    stored as fp16 scaled by a power of two chosen per task from the largest
-//    input magnitude: the QK^T product then carries 11 mantissa bits instead
-//    of bf16's 8 (the temporal softmax has only T' terms, so its outputs are
-//    O(1) and rounding the rotated operands would dominate the error), and the
-//    exact power-of-two scale keeps any finite input in fp16 range;
+//  - raw keys (the usual call): within one position every row has the same
+//    (h, w), so the h and w rotations of Q and K cancel in q.k and only the
+//    t range needs turning.  The first ceil16(d_t) dims of Q and K are turned
+//    (t pairs) and stored as fp16 in place; the remaining dims stay the raw
+//    bf16 inputs, whose products are exact.  QK^T then runs fp16 MMAs on the
+//    first k-steps and bf16 MMAs on the rest, into one fp32 accumulator.  The
+//    rotated operands are never rounded to bf16: the temporal softmax has
+//    only T' terms, its outputs are O(1), and such rounding would dominate the
+//    error.  If the turned values leave fp16's comfortable range the task is
+//    redone with all dims in fp16 under a power-of-two scale;
+//  - keys that come rotated: Q is turned in full, both are stored as fp16
+//    scaled by powers of two, and QK^T runs fp16 MMAs throughout;
 //  - S = Q K^T (fp16) and O = P V (bf16) on the m16n8k16 tensor-core path with
 //    fp32 accumulation; O staged through shared memory for 16-byte row stores.
 #pragma once
@@ -155,27 +161,44 @@ __device__ __forceinline__ int fp16_rescale_exponent(float m) {
     return max(-60, min(60, 13 - e));
 }
 
-// RoPE + fp16 in place for the T rows of one staged operand (raw bf16 rows
-// in shared memory).  Scale 1 unless the largest rotated magnitude is out of
-// fp16's comfortable range; then the rows are read again from global memory
-// and redone with a power-of-two scale, whose exponent is returned.
+// A bf16 pair as packed fp16 times a power of two (no rotation); m tracks the
+// largest magnitude of the unscaled values.
+__device__ __forceinline__ uint32_t cvt_f16_max(uint32_t packed_bf16, float &m) {
+    const float2 x = unpack_bf16x2(packed_bf16);
+    m = fmax3(m, fabsf(x.x), fabsf(x.y));
+    return pack_f16x2(x.x, x.y);
+}
+
+__device__ __forceinline__ uint32_t cvt_f16(uint32_t packed_bf16, float sc) {
+    const float2 x = unpack_bf16x2(packed_bf16);
+    return pack_f16x2(x.x * sc, x.y * sc);
+}
+
+// RoPE (when kRotate; keys that come rotated are only converted) + fp16 in
+// place for the T rows of one staged operand (raw bf16 rows in shared
+// memory).  Scale 1 unless the largest magnitude is out of fp16's
+// comfortable range; then the rows are read again from global memory and
+// redone with a power-of-two scale, whose exponent is returned.
 template <bool kRotate>
 __device__ __forceinline__ int rotate_to_f16(uint8_t *tile, const __nv_bfloat16 *src, size_t base,
                                              size_t tstride, int T, int rlane, int cch,
                                              const float2 (&cs_fixed)[4], const bool (&is_t)[4],
-                                             const float2 *t_tab, bool rotate) {
+                                             const float2 *t_tab) {
     // t pairs: the block's shared copy of the t section (entry j*T + t);
     // h and w pairs: fixed for the task
     auto angle = [&](int r, int e) -> float2 {
-        if (!rotate) return make_float2(1.f, 0.f);
         return is_t[e] ? t_tab[(cch * 4 + e) * T + r] : cs_fixed[e];
     };
     float mx = 0.f;
     for (int r = rlane; r < T; r += 2) {
         uint4 *p = reinterpret_cast<uint4 *>(tile + swz(r, cch));
         const uint4 x = *p;
-        *p = make_uint4(rot_f16_max(x.x, angle(r, 0), mx), rot_f16_max(x.y, angle(r, 1), mx),
-                        rot_f16_max(x.z, angle(r, 2), mx), rot_f16_max(x.w, angle(r, 3), mx));
+        if constexpr (kRotate)
+            *p = make_uint4(rot_f16_max(x.x, angle(r, 0), mx), rot_f16_max(x.y, angle(r, 1), mx),
+                            rot_f16_max(x.z, angle(r, 2), mx), rot_f16_max(x.w, angle(r, 3), mx));
+        else
+            *p = make_uint4(cvt_f16_max(x.x, mx), cvt_f16_max(x.y, mx), cvt_f16_max(x.z, mx),
+                            cvt_f16_max(x.w, mx));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -184,19 +207,54 @@ __device__ __forceinline__ int rotate_to_f16(uint8_t *tile, const __nv_bfloat16 
     const float sc = pow2f(ex);
     for (int r = rlane; r < T; r += 2) {
         const uint4 x = ldg_stream(src + base + r * tstride + cch * 8);
-        float2 c[4];
+        if constexpr (kRotate) {
+            float2 c[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            c[e] = angle(r, e);
-            c[e] = make_float2(c[e].x * sc, c[e].y * sc);
+            for (int e = 0; e < 4; ++e) {
+                c[e] = angle(r, e);
+                c[e] = make_float2(c[e].x * sc, c[e].y * sc);
+            }
+            *reinterpret_cast<uint4 *>(tile + swz(r, cch)) =
+                make_uint4(rot_f16(x.x, c[0]), rot_f16(x.y, c[1]), rot_f16(x.z, c[2]), rot_f16(x.w, c[3]));
+        } else {
+            *reinterpret_cast<uint4 *>(tile + swz(r, cch)) =
+                make_uint4(cvt_f16(x.x, sc), cvt_f16(x.y, sc), cvt_f16(x.z, sc), cvt_f16(x.w, sc));
         }
-        *reinterpret_cast<uint4 *>(tile + swz(r, cch)) =
-            make_uint4(rot_f16(x.x, c[0]), rot_f16(x.y, c[1]), rot_f16(x.z, c[2]), rot_f16(x.w, c[3]));
     }
     return ex;
 }
 
-template <int MAXT>
+// Raw keys: the first nc 16-byte chunks of every Q and K row (dims 0 .. 8nc-1,
+// nc = ceil16(d_t) / 8) turned by their t angles (pairs past the t range are
+// kept) and stored as unscaled fp16 in place.  Lane (rr, cc) = (lane / nc,
+// lane % nc) takes chunk cc of rows rr, rr + rpi, ...  Returns the largest
+// magnitude written (for the fp16 range check).
+__device__ __forceinline__ float turn_t_region(uint8_t *qt, uint8_t *kt, int T, int lane, int nc, int rpi,
+                                               int pe_t, const float2 *t_tab) {
+    float mx = 0.f;
+    if (lane >= rpi * nc) return mx;
+    const int rr = lane / nc;
+    const int cc = lane - rr * nc;
+    for (int r = rr; r < T; r += rpi) {
+        uint4 *pq = reinterpret_cast<uint4 *>(qt + swz(r, cc));
+        uint4 *pk = reinterpret_cast<uint4 *>(kt + swz(r, cc));
+        const uint4 vq = *pq, vk = *pk;
+        float2 c[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int p = cc * 4 + e;
+            c[e] = p < pe_t ? t_tab[p * T + r] : make_float2(1.f, 0.f);
+        }
+        *pq = make_uint4(rot_f16_max(vq.x, c[0], mx), rot_f16_max(vq.y, c[1], mx),
+                         rot_f16_max(vq.z, c[2], mx), rot_f16_max(vq.w, c[3], mx));
+        *pk = make_uint4(rot_f16_max(vk.x, c[0], mx), rot_f16_max(vk.y, c[1], mx),
+                         rot_f16_max(vk.z, c[2], mx), rot_f16_max(vk.w, c[3], mx));
+    }
+    return mx;
+}
+
+// kRawK: k holds raw keys (a.rope_k == 1); otherwise the keys come rotated.
+template <int MAXT, bool kRawK>
 __global__ void __launch_bounds__(Cfg<MAXT>::kMaxWarps * 32)
 temporal_kernel(const __grid_constant__ TemporalArgs a) {
     constexpr int NP = MAXT / 16;   // pairs of n8 key tiles and k16 key steps
@@ -234,6 +292,11 @@ temporal_kernel(const __grid_constant__ TemporalArgs a) {
     const int rlane = lane >> 4;
     const int tl = T - 1;
     const int n_mt = (T + 15) >> 4;
+    // raw keys: the fp16 region is the first nc chunks (ceil16(d_t) dims),
+    // i.e. the first kk16 k-steps of QK^T; rpi rows per pass of the warp
+    const int nc = ((2 * a.rp.pe_t + 15) / 16) * 2;
+    const int kk16 = nc / 2;
+    const int rpi = nc > 0 ? 32 / nc : 32;
 
     for (; task < total; task += stride) {
         const long long bh = task / a.HW;
@@ -258,14 +321,41 @@ temporal_kernel(const __grid_constant__ TemporalArgs a) {
         for (int e = 0; e < 4; ++e) {
             const int p = cch * 4 + e;
             is_t[e] = p < a.rp.pe_t;
-            cs_fixed[e] = is_t[e] ? make_float2(1.f, 0.f) : a.rope_tab[table_index(a.rp, p, 0, h, w)];
+            // h and w angles matter only when Q is turned in full (keys come rotated)
+            cs_fixed[e] = is_t[e] || kRawK ? make_float2(1.f, 0.f)
+                                            : a.rope_tab[table_index(a.rp, p, 0, h, w)];
         }
         cp_async_wait<0>();
         __syncwarp();
-        const int eq = rotate_to_f16<true>(sq, a.q, base, tstride, T, rlane, cch, cs_fixed, is_t, t_tab,
-                                           true);
-        const int ek = rotate_to_f16<true>(sk, a.k, base, tstride, T, rlane, cch, cs_fixed, is_t, t_tab,
-                                           a.rope_k != 0);
+        int eq = 0, ek = 0;
+        int f16_steps = 8;   // k-steps of QK^T that read fp16 operands; the rest read bf16
+        bool full = !kRawK;
+        if constexpr (kRawK) {
+            float mx = turn_t_region(sq, sk, T, lane, nc, rpi, a.rp.pe_t, t_tab);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (fp16_range_ok(mx)) {
+                f16_steps = kk16;
+            } else {
+                // out of fp16's comfortable range: all dims to fp16 under a
+                // power-of-two scale (t pairs turned, h and w pairs kept).  The
+                // first nc chunks were overwritten: fetch them again.
+                __syncwarp();
+                if (cch < nc) {
+                    for (int r = rlane; r < T; r += 2) {
+                        const size_t gofs = base + r * tstride + cch * 8;
+                        *reinterpret_cast<uint4 *>(sq + swz(r, cch)) = ldg_stream(a.q + gofs);
+                        *reinterpret_cast<uint4 *>(sk + swz(r, cch)) = ldg_stream(a.k + gofs);
+                    }
+                }
+                full = true;
+            }
+            __syncwarp();
+        }
+        if (full) {
+            eq = rotate_to_f16<true>(sq, a.q, base, tstride, T, rlane, cch, cs_fixed, is_t, t_tab);
+            ek = rotate_to_f16<kRawK>(sk, a.k, base, tstride, T, rlane, cch, cs_fixed, is_t, t_tab);
+        }
         const float scale_log2 = a.scale_log2 * pow2f(-(eq + ek));
         __syncwarp();
 
@@ -290,10 +380,18 @@ temporal_kernel(const __grid_constant__ TemporalArgs a) {
                         uint32_t b0, b1, b2, b3;
                         const int krow = min(np * 16 + (lane & 7) + ((lane >> 4) << 3), tl);
                         ldsm_x4(ak + swz(krow, kk * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
+                        if (kk < f16_steps) {
 #pragma unroll
-                        for (int m = 0; m < MG; ++m) {
-                            mma_f16(sacc[m][2 * np], af[m][0], af[m][1], af[m][2], af[m][3], b0, b1);
-                            mma_f16(sacc[m][2 * np + 1], af[m][0], af[m][1], af[m][2], af[m][3], b2, b3);
+                            for (int m = 0; m < MG; ++m) {
+                                mma_f16(sacc[m][2 * np], af[m][0], af[m][1], af[m][2], af[m][3], b0, b1);
+                                mma_f16(sacc[m][2 * np + 1], af[m][0], af[m][1], af[m][2], af[m][3], b2, b3);
+                            }
+                        } else {
+#pragma unroll
+                            for (int m = 0; m < MG; ++m) {
+                                mma_bf16(sacc[m][2 * np], af[m][0], af[m][1], af[m][2], af[m][3], b0, b1);
+                                mma_bf16(sacc[m][2 * np + 1], af[m][0], af[m][1], af[m][2], af[m][3], b2, b3);
+                            }
                         }
                     }
                 }

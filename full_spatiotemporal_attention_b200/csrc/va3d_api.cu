@@ -273,7 +273,7 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
     return launch_status();
 }
 
-template <int MAXT>
+template <int MAXT, bool kRawK>
 int launch_temporal_t(const tp::TemporalArgs &a, cudaStream_t st) {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -288,13 +288,13 @@ int launch_temporal_t(const tp::TemporalArgs &a, cudaStream_t st) {
     const int warps = std::max(1, std::min(tp::Cfg<MAXT>::kMaxWarps, budget / warp_bytes));
     const int smem = table_bytes + warps * warp_bytes;
     const int per_sm = std::max(1, std::min(4, (216 * 1024) / smem));
-    if (cudaFuncSetAttribute(tp::temporal_kernel<MAXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(tp::temporal_kernel<MAXT, kRawK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return VA3D_ERR_CUDA;
     const long long tasks = static_cast<long long>(a.BH) * a.HW;
     const long long need = (tasks + warps - 1) / warps;
     const long long blocks = std::min<long long>(need, static_cast<long long>(sms) * per_sm);
-    tp::temporal_kernel<MAXT><<<static_cast<unsigned>(blocks), warps * 32, smem, st>>>(a);
+    tp::temporal_kernel<MAXT, kRawK><<<static_cast<unsigned>(blocks), warps * 32, smem, st>>>(a);
     return launch_status();
 }
 
@@ -315,8 +315,9 @@ int launch_temporal(const void *q, const void *k, bool k_rotated, const void *v,
     a.rope_k = k_rotated ? 0 : 1;
     a.rope_tab = tab;
     a.rp = rp;
-    if (rp.T <= 32) return launch_temporal_t<32>(a, st);
-    return launch_temporal_t<64>(a, st);
+    if (rp.T <= 32)
+        return k_rotated ? launch_temporal_t<32, false>(a, st) : launch_temporal_t<32, true>(a, st);
+    return k_rotated ? launch_temporal_t<64, false>(a, st) : launch_temporal_t<64, true>(a, st);
 }
 
 // Shared front half of the two attention entry points: checks, workspace

@@ -190,6 +190,29 @@ def test_factorised_sampled_rows_full_size(va):
         check(got, ref, f"{mode} c81f720")
 
 
+def _scale_bits(bits, k):
+    """bf16 bit patterns times 2^k, exactly (exponent field + k; zeros kept)."""
+    b = bits.astype(np.int32)
+    nz = (b & 0x7FFF) != 0
+    b = np.where(nz, b + (k << 7), b)
+    return b.astype(np.uint16)
+
+
+@pytest.mark.parametrize("k", [-14, -8, 8, 14])
+def test_temporal_pass_at_extreme_magnitudes(va, k):
+    """Queries times 2^k and keys times 2^-k leave every logit exactly as it
+    was while moving the turned values out of fp16's comfortable range
+    (k = +-14: the power-of-two-scaled path) or to its edges (k = +-8: the
+    unscaled path with small operands near fp16's subnormals)."""
+    w = si.WORKLOADS["c17f480"]
+    q, kk, v = si.qkv(w)
+    q, kk = _scale_bits(q, k), _scale_bits(kk, -k)
+    _, ot = va.attn_factorized_fwd(dev(q), dev(kk), dev(v), vgrid(va, w), spatial=False)
+    ref = oracle.attention(q, kk, v, ogrid(w), mode="temporal")
+    check(host(ot).reshape(ref.shape), ref, f"temporal 2^{k}")
+    assert va.device_error() == 0
+
+
 def test_factorised_single_pass_outputs(va):
     w = si.WORKLOADS["tiny"]
     q, k, v = (dev(x) for x in si.qkv(w))
