@@ -11,10 +11,13 @@ angle table, and the fused Q-RoPE + attention kernel.  Inputs are resident
 in HBM before timing; Q, K, V and O together (403 MB) exceed the 126 MB L2.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--parallel replicas|ulysses]
 
-For N > 1 launch one process per GPU with torch.distributed.run; every rank
-runs an independent replica of the workload (weak scaling, no collective on
-the data path) and rank 0 prints one JSON line.
+For N > 1 launch one process per GPU with torch.distributed.run; by default
+every rank runs an independent replica of the workload (weak scaling, no
+collective on the data path) and rank 0 prints one JSON line.  With
+--parallel ulysses the ranks split one sequence (strong scaling): token
+slices are exchanged for head groups over peer memory and back.
 """
 import argparse
 import hashlib
@@ -45,6 +48,10 @@ def parse_args():
     p.add_argument("--no-extras", action="store_true", help="skip the secondary measurements")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
+    p.add_argument("--parallel", choices=["replicas", "ulysses"], default="replicas",
+                   help="N > 1: independent replicas per rank (default), or one sequence split "
+                        "over the ranks with Ulysses context parallelism (strong scaling; heads "
+                        "and tokens must divide by N)")
     p.add_argument("--case", choices=["temporal720", "spatial720", "window720", "cross720"],
                    help="run only this secondary kernel (warm-up + --steps launches, one "
                         "JSON line); a small, single-kernel command for profilers")
@@ -511,7 +518,140 @@ def extras(va, device, stream, peak_tf, peak_gbs):
                        "frac_of_hbm": round(b_x / x_ms / 1e6 / peak_gbs, 4)}
     del q, k, v, o, ws
     torch.cuda.empty_cache()
+
+    # the context-parallel step on one rank (its exchange kernels then copy
+    # locally): the 480p clip, scatter (Q, K, V with the key RoPE) and gather
+    from full_spatiotemporal_attention_b200.ulysses import UlyssesAttention
+    w = si.WORKLOADS["c81f480"]
+    q, k, v = (to_dev(x, device) for x in si.qkv(w))
+    g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    ua = UlyssesAttention(g, w.batch, w.heads, world=1, rank=0, device=device)
+    _, u_ms = timed_loop(ev_pair(lambda: ua(q, k, v)), 5, 3, 1, device)
+    _, s_ms = timed_loop(ev_pair(lambda: ua.scatter(q, k, v)), 20, 3, 1, device)
+    _, g_ms = timed_loop(ev_pair(ua.gather), 20, 3, 1, device)
+    torch.cuda.synchronize()
+    ua.close()
+    tb = w.batch * w.heads * w.N * HEAD_DIM * 2
+    out["ulysses480_1rank"] = {
+        "step_ms": round(u_ms, 4), "tflops": round(full_flops(w) / u_ms / 1e9, 1),
+        "scatter_ms": round(s_ms, 4), "scatter_gbs": round(6 * tb / s_ms / 1e6, 1),
+        "scatter_frac_hbm": round(6 * tb / s_ms / 1e6 / peak_gbs, 4),
+        "gather_ms": round(g_ms, 4), "gather_gbs": round(2 * tb / g_ms / 1e6, 1),
+        "gather_frac_hbm": round(2 * tb / g_ms / 1e6 / peak_gbs, 4)}
+    del q, k, v, ua
+    torch.cuda.empty_cache()
     return out
+
+
+def bench_ulysses(args, rank, world, local):
+    """One sequence of the workload split over the ranks (Ulysses context
+    parallelism through peer memory): each rank holds a contiguous token
+    slice of every head; a step scatters it, runs full attention on whole
+    sequences of its heads and gathers its slice of the output."""
+    import numpy as np
+    import torch
+    import full_spatiotemporal_attention_b200 as va
+    from full_spatiotemporal_attention_b200.ulysses import UlyssesAttention
+    import seeded_inputs as si
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = si.WORKLOADS[args.workload]
+    g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    ua = UlyssesAttention(g, w.batch, w.heads, world=world, rank=rank, device=device)
+    t0, t1 = ua.plan.token_range
+    host = [np.ascontiguousarray(x[:, :, t0:t1]) for x in si.qkv(w)]
+    q, k, v = (to_dev(x, device) for x in host)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        ua(q, k, v)
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.5)
+    window = []
+    step_ms, _ = timed_loop(step, args.steps, args.warmup, world, device, window=window)
+    clocks = sampler.stop(*window)
+    step_ms = max_over_ranks(step_ms, world, device)
+
+    # the three steps alone (every rank runs the same sequence)
+    def phase(fn):
+        def run(i):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            return a, b
+        return run
+    n = max(args.steps // 2, 5)
+    _, sc_ms = timed_loop(phase(lambda: ua.scatter(q, k, v)), n, 3, world, device)
+    _, at_ms = timed_loop(phase(ua.attend), n, 3, world, device)
+    _, ga_ms = timed_loop(phase(ua.gather), n, 3, world, device)
+    sc_ms, at_ms, ga_ms = (max_over_ranks(x, world, device) for x in (sc_ms, at_ms, ga_ms))
+
+    # end to end: this rank's slice from pinned host memory, its output slice back
+    qh, kh, vh = (torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in host)
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd = (torch.empty_like(q) for _ in range(3))
+
+    def e2e_step(i):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        oh.copy_(ua(qd, kd, vd), non_blocking=True)
+    e2e_ms, _ = timed_loop(e2e_step, args.e2e_steps, 3, world, device)
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
+    torch.cuda.synchronize()
+    assert va.device_error() == 0, "a peer wait gave up"
+    ua.close(barrier=(lambda: barrier(world)))
+
+    flops = full_flops(w)
+    peak_tf, peak_gbs, peak_src = peaks()
+    shard = w.batch * w.heads * (w.N // world) * HEAD_DIM * 2   # one tensor's slice per rank
+    attn_flops_rank = flops / world
+    cfg = job_config(w, world)
+    cfg.update(global_batch=w.batch,
+               parallelism=f"ulysses x{world} (token slices <-> head groups over peer memory)")
+    return {
+        "metric": METRIC,
+        "value": round(flops / (step_ms / 1e3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded splitmix64 + Box-Muller bf16 N(0,1))",
+        "config": cfg,
+        "pct_of_peak": round(100.0 * flops / (step_ms / 1e3) / 1e12 / world / peak_tf, 2),
+        "e2e": {"value": round(flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": 3 * shard,
+                "d2h_bytes_per_step": shard},
+        "gpu_launches": 6 * args.steps,
+        "roofline": {"bound": "tensor", "achieved": round(attn_flops_rank / (at_ms / 1e3) / 1e12, 2),
+                     "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(attn_flops_rank / (at_ms / 1e3) / 1e12 / peak_tf, 4),
+                     "traffic": None, "kernel": "attn_fwd_kernel",
+                     "peak_source": f"{peak_src} bf16 dense (burst)", "kernel_ms": round(at_ms, 4)},
+        "exchange": {
+            "scatter_ms": round(sc_ms, 4), "gather_ms": round(ga_ms, 4),
+            # per rank: Q, K, V slices read and written; O slices read and written
+            "scatter_gbs": round(6 * shard / (sc_ms / 1e3) / 1e9, 1),
+            "gather_gbs": round(2 * shard / (ga_ms / 1e3) / 1e9, 1),
+            "bytes_to_peers_per_step": int(4 * shard * (world - 1) / world),
+            "peak_gbs_local": peak_gbs},
+        "clocks": clocks,
+    }
 
 
 def run_case(args):
@@ -606,7 +746,7 @@ def main():
         print(json.dumps(run_case(args)), flush=True)
         return
     rank, world, local = init_dist("nccl")
-    line = bench_ours(args, rank, world, local)
+    line = (bench_ulysses if args.parallel == "ulysses" else bench_ours)(args, rank, world, local)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

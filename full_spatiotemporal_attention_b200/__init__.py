@@ -13,6 +13,9 @@ Entry points (same names as the C ABI):
 * ``attn_factorized_fwd(q, k, v, grid)``    spatial and temporal passes
 * ``attn_cross_fwd(q, k, v)``               video-to-text cross-attention (no RoPE)
 * ``attn_window_fwd(q, k, v, grid, window)`` local 3D-window attention
+* ``ulysses_scatter / ulysses_gather / ulysses_wait`` and the region / IPC
+  calls: the exchange steps of Ulysses context parallelism (composed by
+  ``ulysses.UlyssesAttention``)
 * ``grid_from_video(frames, height, width)``  token grid of a clip
 * ``workspace_bytes(...)``, ``device_error()``
 """
@@ -32,7 +35,9 @@ SYMBOLS = ("va3d_status_string", "va3d_version", "va3d_grid_from_video",
            "va3d_workspace_bytes", "rope3d_apply", "attn3d_full_fwd",
            "attn_factorized_fwd", "va3d_device_error", "attn3d_full_fwd_noalloc",
            "va3d_cross_workspace_bytes", "attn_cross_fwd", "attn_window_fwd",
-           "va3d_watchdog_selftest")
+           "va3d_watchdog_selftest", "va3d_ulysses_region_bytes", "va3d_ulysses_offsets",
+           "va3d_region_alloc", "va3d_region_free", "va3d_ipc_export", "va3d_ipc_open",
+           "va3d_ipc_close", "va3d_ulysses_scatter", "va3d_ulysses_gather", "va3d_ulysses_wait")
 
 
 class VA3DError(RuntimeError):
@@ -89,6 +94,18 @@ def _load():
     lib.va3d_cross_workspace_bytes.restype = sz
     lib.attn_cross_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
     lib.attn_window_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, gp, i, i, i, f, u, vp, sz, vp]
+    szp, vpp = ctypes.POINTER(sz), ctypes.POINTER(vp)
+    lib.va3d_ulysses_region_bytes.argtypes = [i, i, i, i, i]
+    lib.va3d_ulysses_region_bytes.restype = sz
+    lib.va3d_ulysses_offsets.argtypes = [i, i, i, i, i, szp, szp, szp, szp]
+    lib.va3d_region_alloc.argtypes = [sz, vpp]
+    lib.va3d_region_free.argtypes = [vp]
+    lib.va3d_ipc_export.argtypes = [vp, ctypes.c_char_p]
+    lib.va3d_ipc_open.argtypes = [ctypes.c_char_p, vpp]
+    lib.va3d_ipc_close.argtypes = [vp]
+    lib.va3d_ulysses_scatter.argtypes = [vp, vp, vp, vpp, i, i, i, i, i, i, gp, u, vp]
+    lib.va3d_ulysses_gather.argtypes = [vp, vpp, i, i, i, i, i, i, vp]
+    lib.va3d_ulysses_wait.argtypes = [vp, i, ctypes.c_ulonglong, i, i, i, i, i, vp]
     return lib
 
 
@@ -316,6 +333,128 @@ def attn_cross_fwd(q, k, v, *, scale=None, return_lse=False, out=None, lse=None,
     if rc != VA3D_OK:
         raise VA3DError("attn_cross_fwd", rc)
     return (out, lse) if (return_lse or lse is not None) else out
+
+
+# ------------------------------------------- Ulysses context parallelism
+
+IPC_HANDLE_BYTES = 64
+PHASE_SCATTER, PHASE_GATHER = 0, 1
+
+
+def ulysses_region_bytes(B, heads, N, world):
+    """Bytes of one rank's exchange region (0 if the sizes are not supported)."""
+    return int(lib.va3d_ulysses_region_bytes(B, heads, N, HEAD_DIM, world))
+
+
+def ulysses_offsets(B, heads, N, world):
+    """(off_q, off_k, off_v, off_o): byte offsets of Qh, Kh, Vh and the O shard."""
+    offs = [ctypes.c_size_t() for _ in range(4)]
+    rc = lib.va3d_ulysses_offsets(B, heads, N, HEAD_DIM, world, *(ctypes.byref(o) for o in offs))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ulysses_offsets", rc)
+    return tuple(int(o.value) for o in offs)
+
+
+def region_alloc(nbytes):
+    """Device memory (cudaMalloc, zeroed) on the current device; returns its address."""
+    p = ctypes.c_void_p()
+    rc = lib.va3d_region_alloc(int(nbytes), ctypes.byref(p))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_region_alloc", rc)
+    return int(p.value)
+
+
+def region_free(ptr):
+    rc = lib.va3d_region_free(ctypes.c_void_p(ptr))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_region_free", rc)
+
+
+def ipc_export(ptr):
+    """CUDA IPC handle of a region, as bytes."""
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    rc = lib.va3d_ipc_export(ctypes.c_void_p(ptr), buf)
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ipc_export", rc)
+    return buf.raw
+
+
+def ipc_open(handle):
+    """Map a peer's region from its handle; returns the address in this process."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {IPC_HANDLE_BYTES} bytes, got {len(handle)}")
+    p = ctypes.c_void_p()
+    rc = lib.va3d_ipc_open(bytes(handle), ctypes.byref(p))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ipc_open", rc)
+    return int(p.value)
+
+
+def ipc_close(ptr):
+    rc = lib.va3d_ipc_close(ctypes.c_void_p(ptr))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ipc_close", rc)
+
+
+def _ptr_array(regions):
+    return (ctypes.c_void_p * len(regions))(*[ctypes.c_void_p(int(r)) for r in regions])
+
+
+def ulysses_scatter(q, k, v, regions, rank, grid, *, k_rotated=False):
+    """Send this rank's token slice q, k, v [B, heads, N/world, 128] to every
+    rank's region (world = len(regions)); keys turned at their global
+    positions unless k_rotated."""
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    B, H, n_loc, D = q.shape
+    world = len(regions)
+    rc = lib.va3d_ulysses_scatter(_ptr(q), _ptr(k), _ptr(v), _ptr_array(regions), world, rank, B, H,
+                                  n_loc * world, D, ctypes.byref(grid),
+                                  VA3D_K_ROTATED if k_rotated else 0, _stream(q))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ulysses_scatter", rc)
+
+
+def ulysses_gather(o_heads, regions, rank, heads):
+    """Send this rank's attention output o_heads [B, heads/world, N, 128] back
+    as token slices into every rank's O shard."""
+    _check(o_heads, "o_heads")
+    B, hpw, N, D = o_heads.shape
+    world = len(regions)
+    if hpw * world != heads:
+        raise ValueError(f"o_heads holds {hpw} heads, expected {heads} / {world}")
+    rc = lib.va3d_ulysses_gather(_ptr(o_heads), _ptr_array(regions), world, rank, B, heads, N, D,
+                                 _stream(o_heads))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ulysses_gather", rc)
+
+
+def ulysses_wait(region, phase, epoch, world, B, heads, N, device=None):
+    """Stream-ordered, bounded wait for every peer's signals of call `epoch`."""
+    torch = _torch()
+    st = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    rc = lib.va3d_ulysses_wait(ctypes.c_void_p(region), phase, int(epoch), world, B, heads, N,
+                               HEAD_DIM, st)
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ulysses_wait", rc)
+
+
+class _DeviceMemory:
+    """__cuda_array_interface__ of a stretch of a region, for a zero-copy tensor view."""
+
+    def __init__(self, ptr, shape):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": "<i2",
+                                         "data": (int(ptr), False), "version": 3,
+                                         "strides": None}
+
+
+def region_view(ptr, offset, shape, device):
+    """bf16 tensor of `shape` over region memory at ptr + offset (no copy; the
+    region must outlive it)."""
+    torch = _torch()
+    t = torch.as_tensor(_DeviceMemory(ptr + offset, shape), device=device)
+    return t.view(torch.bfloat16)
 
 
 def watchdog_selftest():

@@ -18,6 +18,7 @@
 #include "attn_sm100.cuh"
 #include "attn_temporal.cuh"
 #include "selftest.cuh"
+#include "ulysses.cuh"
 
 using namespace va3d;
 
@@ -149,6 +150,25 @@ int make_map(CUtensorMap *map, const void *base, int N, int BH, int box_rows) {
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? VA3D_OK : VA3D_ERR_CUDA;
+}
+
+// Shapes of a Ulysses exchange: the attention limits on whole sequences
+// (B, heads/world, N) and on the local slices (B, heads, N/world).
+int check_ulysses(int B, int heads, int N, int head_dim, int world) {
+    if (world < 1 || world > cp::kMaxWorld) return VA3D_ERR_UNSUPPORTED;
+    int rc;
+    if ((rc = check_sizes(B, heads, N, head_dim)) != VA3D_OK) return rc;
+    if (heads % world != 0 || N % world != 0) return VA3D_ERR_UNSUPPORTED;
+    return VA3D_OK;
+}
+
+int check_regions(void *const *regions, int world, int rank) {
+    if (regions == nullptr || rank < 0 || rank >= world) return VA3D_ERR_INVALID;
+    for (int j = 0; j < world; ++j) {
+        if (regions[j] == nullptr) return VA3D_ERR_INVALID;
+        if ((reinterpret_cast<uintptr_t>(regions[j]) & 255u) != 0) return VA3D_ERR_ALIGNMENT;
+    }
+    return VA3D_OK;
 }
 
 int launch_status() {
@@ -539,6 +559,143 @@ int va3d_device_error(int reset) {
     return value;
 }
 
+
+size_t va3d_ulysses_region_bytes(int B, int heads, int N, int head_dim, int world) {
+    if (check_ulysses(B, heads, N, head_dim, world) != VA3D_OK) return 0;
+    return cp::region_layout(B, heads, N, world).bytes;
+}
+
+int va3d_ulysses_offsets(int B, int heads, int N, int head_dim, int world, size_t *off_q,
+                         size_t *off_k, size_t *off_v, size_t *off_o) {
+    int rc;
+    if ((rc = check_ulysses(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
+    if (off_q == nullptr || off_k == nullptr || off_v == nullptr || off_o == nullptr)
+        return VA3D_ERR_INVALID;
+    const cp::Layout l = cp::region_layout(B, heads, N, world);
+    *off_q = l.q;
+    *off_k = l.k;
+    *off_v = l.v;
+    *off_o = l.o;
+    return VA3D_OK;
+}
+
+int va3d_region_alloc(size_t bytes, void **ptr) {
+    if (bytes == 0 || ptr == nullptr) return VA3D_ERR_INVALID;
+    *ptr = nullptr;
+    void *p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return VA3D_ERR_CUDA;
+    if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        cudaFree(p);
+        return VA3D_ERR_CUDA;
+    }
+    *ptr = p;
+    return VA3D_OK;
+}
+
+int va3d_region_free(void *ptr) {
+    if (ptr == nullptr) return VA3D_ERR_INVALID;
+    return cudaFree(ptr) == cudaSuccess ? VA3D_OK : VA3D_ERR_CUDA;
+}
+
+int va3d_ipc_export(const void *region, unsigned char *handle) {
+    static_assert(sizeof(cudaIpcMemHandle_t) == VA3D_IPC_HANDLE_BYTES, "IPC handle size");
+    if (region == nullptr || handle == nullptr) return VA3D_ERR_INVALID;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, const_cast<void *>(region)) != cudaSuccess) return VA3D_ERR_CUDA;
+    std::memcpy(handle, &h, sizeof h);
+    return VA3D_OK;
+}
+
+int va3d_ipc_open(const unsigned char *handle, void **ptr) {
+    if (handle == nullptr || ptr == nullptr) return VA3D_ERR_INVALID;
+    *ptr = nullptr;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof h);
+    void *p = nullptr;
+    if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return VA3D_ERR_CUDA;
+    *ptr = p;
+    return VA3D_OK;
+}
+
+int va3d_ipc_close(void *ptr) {
+    if (ptr == nullptr) return VA3D_ERR_INVALID;
+    return cudaIpcCloseMemHandle(ptr) == cudaSuccess ? VA3D_OK : VA3D_ERR_CUDA;
+}
+
+int va3d_ulysses_scatter(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
+                         void *const *regions, int world, int rank, int B, int heads, int N,
+                         int head_dim, const va3d_grid_t *grid, unsigned flags, void *stream) {
+    int rc;
+    if ((rc = check_ulysses(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
+    if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
+    if ((rc = check_regions(regions, world, rank)) != VA3D_OK) return rc;
+    if (q == nullptr || k == nullptr || v == nullptr) return VA3D_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return VA3D_ERR_ALIGNMENT;
+    if (flags & ~static_cast<unsigned>(VA3D_K_ROTATED)) return VA3D_ERR_INVALID;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    const cp::Layout l = cp::region_layout(B, heads, N, world);
+    cp::ScatterArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.q = static_cast<const uint4 *>(static_cast<const void *>(q));
+    a.k = static_cast<const uint4 *>(static_cast<const void *>(k));
+    a.v = static_cast<const uint4 *>(static_cast<const void *>(v));
+    for (int j = 0; j < world; ++j) a.region[j] = static_cast<uint8_t *>(regions[j]);
+    a.off_q = l.q;
+    a.off_k = l.k;
+    a.off_v = l.v;
+    a.world = world;
+    a.rank = rank;
+    a.B = B;
+    a.heads = heads;
+    a.hpw = heads / world;
+    a.N = N;
+    a.n_loc = N / world;
+    a.rotate_k = (flags & VA3D_K_ROTATED) ? 0 : 1;
+    const int blocks = cp::copy_blocks(a.n_loc);
+    cp::ulysses_scatter_kernel<<<blocks, cp::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        a, make_rope_params(grid));
+    return launch_status();
+}
+
+int va3d_ulysses_gather(const va3d_bf16 *o_heads, void *const *regions, int world, int rank,
+                        int B, int heads, int N, int head_dim, void *stream) {
+    int rc;
+    if ((rc = check_ulysses(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
+    if ((rc = check_regions(regions, world, rank)) != VA3D_OK) return rc;
+    if (o_heads == nullptr) return VA3D_ERR_INVALID;
+    if (!aligned16(o_heads)) return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    cp::GatherArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.o = static_cast<const uint4 *>(static_cast<const void *>(o_heads));
+    for (int j = 0; j < world; ++j) a.region[j] = static_cast<uint8_t *>(regions[j]);
+    a.off_o = cp::region_layout(B, heads, N, world).o;
+    a.world = world;
+    a.rank = rank;
+    a.B = B;
+    a.heads = heads;
+    a.hpw = heads / world;
+    a.N = N;
+    a.n_loc = N / world;
+    const int blocks = cp::copy_blocks(N);
+    cp::ulysses_gather_kernel<<<blocks, cp::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+int va3d_ulysses_wait(const void *region, int phase, unsigned long long epoch, int world, int B,
+                      int heads, int N, int head_dim, void *stream) {
+    int rc;
+    if ((rc = check_ulysses(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
+    if (region == nullptr || (phase != cp::kScatter && phase != cp::kGather) || epoch == 0)
+        return VA3D_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(region) & 255u) != 0) return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    const int blocks = cp::copy_blocks(phase == cp::kScatter ? N / world : N);
+    const unsigned long long expected = epoch * static_cast<unsigned long long>(world) * blocks;
+    cp::ulysses_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const unsigned long long *>(region), phase, expected);
+    return launch_status();
+}
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

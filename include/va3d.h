@@ -88,7 +88,8 @@ enum {
     VA3D_DEVERR_TIMEOUT_LOAD = 1,     /* a wait in the tile-loading role timed out */
     VA3D_DEVERR_TIMEOUT_MMA = 2,      /* a wait in the MMA-issuing role timed out */
     VA3D_DEVERR_TIMEOUT_SOFTMAX = 3,  /* a wait in the softmax role timed out */
-    VA3D_DEVERR_TIMEOUT_SELFTEST = 4  /* the wait of va3d_watchdog_selftest timed out (expected) */
+    VA3D_DEVERR_TIMEOUT_SELFTEST = 4, /* the wait of va3d_watchdog_selftest timed out (expected) */
+    VA3D_DEVERR_TIMEOUT_PEER = 5      /* va3d_ulysses_wait gave up on its peers */
 };
 
 /* Human-readable text of a status code; never NULL. */
@@ -276,6 +277,102 @@ int va3d_watchdog_selftest(void *stream);
  * word is cleared afterwards.  Returns VA3D_ERR_CUDA if it cannot be read.
  */
 int va3d_device_error(int reset);
+
+/* ------------------------------------------------------------------------
+ * Ulysses context parallelism over peer memory (one process per GPU).
+ *
+ * The pages on full 3D attention name context parallelism (Ulysses and
+ * ring) as what long videos turn to (anthology record sota-390, "budget for
+ * that cost"), and note that 3D RoPE needs no exchange under sequence
+ * parallelism because each rank's token coordinates are absolute (handbook
+ * "A video model's architecture", section "Position: RoPE in three
+ * dimensions").  Rank r of `world` holds the contiguous token slice
+ * [r*N/world, (r+1)*N/world) of every head, as [B, heads, N/world, 128].
+ * va3d_ulysses_scatter sends each head group (heads/world heads) with all
+ * its tokens to the rank that owns it, turning keys by their global
+ * positions on the way; attn3d_full_fwd then runs on whole sequences (keys
+ * already rotated, VA3D_K_ROTATED); va3d_ulysses_gather sends each token
+ * slice of the output back.  Transfers are 16-byte stores into the peers'
+ * regions; each copy kernel then signals every peer's counter, and
+ * va3d_ulysses_wait (bounded) orders a rank's next step after its peers'.
+ *
+ * Region (one per rank, device memory from va3d_region_alloc, mapped into
+ * every rank with the IPC calls): a 256-byte header holding two u64
+ * counters (scatter, gather; zero at allocation and never reset), then
+ * Qh, Kh, Vh, each [B, heads/world, N, 128] bf16 (this rank's heads, all
+ * tokens), then the O shard [B, heads, N/world, 128] bf16 (all heads, this
+ * rank's tokens).  Requirements: 1 <= world <= 8, heads and N divisible by
+ * world, 0 <= rank < world; the same shapes on every rank.
+ * ---------------------------------------------------------------------- */
+
+#define VA3D_IPC_HANDLE_BYTES 64
+
+/* Bytes of one rank's region; 0 if the sizes are invalid or unsupported. */
+size_t va3d_ulysses_region_bytes(int B, int heads, int N, int head_dim, int world);
+
+/*
+ * Byte offsets of Qh, Kh, Vh and the O shard inside a region (each
+ * 256-byte aligned).  Errors: VA3D_ERR_INVALID, _UNSUPPORTED.
+ */
+int va3d_ulysses_offsets(int B, int heads, int N, int head_dim, int world, size_t *off_q,
+                         size_t *off_k, size_t *off_v, size_t *off_o);
+
+/*
+ * Allocate `bytes` of device memory on the current device with cudaMalloc
+ * and zero it (set-up time, not in a hot call; the counters must start at
+ * zero).  The caller owns it and frees it with va3d_region_free.
+ * Errors: VA3D_ERR_INVALID (bytes == 0 or ptr NULL), _CUDA.
+ */
+int va3d_region_alloc(size_t bytes, void **ptr);
+int va3d_region_free(void *ptr);
+
+/*
+ * CUDA IPC handle (VA3D_IPC_HANDLE_BYTES bytes, written to `handle`) of a
+ * region returned by va3d_region_alloc; va3d_ipc_open maps a peer's region
+ * into this process (peer access enabled lazily) and va3d_ipc_close unmaps
+ * it.  The handle travels between processes as plain bytes.
+ * Errors: VA3D_ERR_INVALID (NULL arguments), _CUDA.
+ */
+int va3d_ipc_export(const void *region, unsigned char *handle);
+int va3d_ipc_open(const unsigned char *handle, void **ptr);
+int va3d_ipc_close(void *ptr);
+
+/*
+ * Scatter this rank's slice: q, k, v are [B, heads, N/world, 128] bf16
+ * (16-byte aligned), `regions` a host array of `world` region pointers
+ * valid in this process, index j = rank j's region (this rank's own at
+ * index `rank`).  Writes rank j's Qh, Kh, Vh rows [rank*N/world,
+ * (rank+1)*N/world) of heads [j*heads/world, (j+1)*heads/world); keys are
+ * turned by 3D RoPE at their global positions unless flags has
+ * VA3D_K_ROTATED.  Then adds, per block of its grid, 1 to every region's
+ * scatter counter.  Asynchronous on `stream`.
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _ALIGNMENT, _DEVICE, _CUDA.
+ */
+int va3d_ulysses_scatter(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
+                         void *const *regions, int world, int rank, int B, int heads, int N,
+                         int head_dim, const va3d_grid_t *grid, unsigned flags, void *stream);
+
+/*
+ * Gather: o_heads is this rank's attention output [B, heads/world, N, 128]
+ * bf16 (16-byte aligned).  Writes, for every rank j, its O shard rows of
+ * heads [rank*heads/world, (rank+1)*heads/world); then adds, per block, 1
+ * to every region's gather counter.  Asynchronous on `stream`.
+ * Errors: as va3d_ulysses_scatter.
+ */
+int va3d_ulysses_gather(const va3d_bf16 *o_heads, void *const *regions, int world, int rank,
+                        int B, int heads, int N, int head_dim, void *stream);
+
+/*
+ * Stream-ordered wait until this rank's counter for `phase` (0 scatter,
+ * 1 gather) has received every peer's signals of call number `epoch`
+ * (1, 2, ...), i.e. reaches epoch * world * blocks of that copy kernel.
+ * Bounded: after 2 s it records VA3D_DEVERR_TIMEOUT_PEER in the device
+ * error word and returns, so a rank that never arrives cannot hang the GPU
+ * (the data read after it is then incomplete; check va3d_device_error).
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _DEVICE, _CUDA.
+ */
+int va3d_ulysses_wait(const void *region, int phase, unsigned long long epoch, int world, int B,
+                      int heads, int N, int head_dim, void *stream);
 
 #ifdef __cplusplus
 }

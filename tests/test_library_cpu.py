@@ -105,8 +105,9 @@ def test_status_strings(va):
 def test_bad_arguments_rejected_before_any_device_call(va):
     lib = va.lib
     g = va.Grid.make(2, 4, 4)
-    buf = ctypes.create_string_buffer(4096 + 16)
-    p = ctypes.c_void_p((ctypes.addressof(buf) + 15) // 16 * 16)
+    # 256-byte aligned, so that p + 16 is 16-byte but never 256-byte aligned
+    buf = ctypes.create_string_buffer(4096 + 256)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256)
     gp = ctypes.byref(g)
     # head_dim other than 128
     assert lib.attn3d_full_fwd(p, p, p, p, None, 1, 2, 32, 64, gp, 0.0, 0, p, 4096, None) == -2
@@ -149,6 +150,61 @@ def test_bad_arguments_rejected_before_any_device_call(va):
     # odd RoPE range
     godd = va.Grid.make(2, 4, 4, dims=(43, 43, 42))
     assert lib.rope3d_apply(p, p, 1, 2, 32, 128, ctypes.byref(godd), None) == -1
+
+
+def test_ulysses_region_layout(va):
+    """Region = 256-byte header, Qh, Kh, Vh [B, heads/P, N, 128] and the O
+    shard [B, heads, N/P, 128], bf16 rows of 256 bytes."""
+    B, H, N, P = 2, 12, 7800, 4
+    head_shard = B * (H // P) * N * 256
+    seq_shard = B * H * (N // P) * 256
+    assert va.ulysses_offsets(B, H, N, P) == (256, 256 + head_shard, 256 + 2 * head_shard,
+                                              256 + 3 * head_shard)
+    assert va.ulysses_region_bytes(B, H, N, P) == 256 + 3 * head_shard + seq_shard
+    # one rank holds everything twice over: whole sequences and its (whole) shard
+    assert va.ulysses_region_bytes(1, 2, 32, 1) == 256 + 4 * 2 * 32 * 256
+    # heads or tokens that do not split, or more ranks than one node holds
+    for args in ((1, 12, 7800, 8), (1, 12, 7801, 4), (1, 16, 32, 9), (1, 16, 32, 0)):
+        assert va.ulysses_region_bytes(*args) == 0
+    with pytest.raises(va.VA3DError):
+        va.ulysses_offsets(1, 12, 7800, 8)
+
+
+def test_ulysses_bad_arguments_rejected_before_any_device_call(va):
+    lib = va.lib
+    g = va.Grid.make(2, 4, 4)
+    gp = ctypes.byref(g)
+    buf = ctypes.create_string_buffer(4096 + 256)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256)
+    regions = (ctypes.c_void_p * 2)(p, p)
+    # heads not divisible by world; tokens not divisible; head_dim; world range
+    assert lib.va3d_ulysses_scatter(p, p, p, regions, 2, 0, 1, 3, 32, 128, gp, 0, None) == -2
+    assert lib.va3d_ulysses_scatter(p, p, p, regions, 2, 0, 1, 2, 32, 64, gp, 0, None) == -2
+    assert lib.va3d_ulysses_scatter(p, p, p, regions, 9, 0, 1, 18, 36, 128, gp, 0, None) == -2
+    assert lib.va3d_ulysses_scatter(p, p, p, regions, 0, 0, 1, 2, 32, 128, gp, 0, None) == -2
+    # grid inconsistent with N; rank out of range; missing region; unknown flag
+    assert lib.va3d_ulysses_scatter(p, p, p, regions, 2, 0, 1, 2, 34, 128, gp, 0, None) == -1
+    assert lib.va3d_ulysses_scatter(p, p, p, regions, 2, 2, 1, 2, 32, 128, gp, 0, None) == -1
+    holes = (ctypes.c_void_p * 2)(p, None)
+    assert lib.va3d_ulysses_scatter(p, p, p, holes, 2, 0, 1, 2, 32, 128, gp, 0, None) == -1
+    assert lib.va3d_ulysses_scatter(p, p, p, regions, 2, 0, 1, 2, 32, 128, gp, 4, None) == -1
+    # a region must be 256-byte aligned, tensors 16-byte aligned
+    odd = (ctypes.c_void_p * 2)(p, ctypes.c_void_p(p.value + 16))
+    assert lib.va3d_ulysses_scatter(p, p, p, odd, 2, 0, 1, 2, 32, 128, gp, 0, None) == -3
+    q = ctypes.c_void_p(p.value + 2)
+    assert lib.va3d_ulysses_scatter(q, p, p, regions, 2, 0, 1, 2, 32, 128, gp, 0, None) == -3
+    assert lib.va3d_ulysses_gather(q, regions, 2, 0, 1, 2, 32, 128, None) == -3
+    assert lib.va3d_ulysses_gather(p, regions, 2, 5, 1, 2, 32, 128, None) == -1
+    # wait: phase, epoch 0, alignment
+    assert lib.va3d_ulysses_wait(p, 2, 1, 2, 1, 2, 32, 128, None) == -1
+    assert lib.va3d_ulysses_wait(p, 0, 0, 2, 1, 2, 32, 128, None) == -1
+    assert lib.va3d_ulysses_wait(ctypes.c_void_p(p.value + 8), 0, 1, 2, 1, 2, 32, 128, None) == -3
+    # set-up calls
+    assert lib.va3d_region_alloc(0, ctypes.byref(ctypes.c_void_p())) == -1
+    assert lib.va3d_ipc_export(None, ctypes.create_string_buffer(64)) == -1
+    assert lib.va3d_ipc_open(None, ctypes.byref(ctypes.c_void_p())) == -1
+    with pytest.raises(ValueError, match="64 bytes"):
+        va.ipc_open(b"short")
 
 
 def test_binding_has_no_cpu_path(va):
