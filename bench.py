@@ -48,10 +48,11 @@ def parse_args():
     p.add_argument("--no-extras", action="store_true", help="skip the secondary measurements")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
-    p.add_argument("--parallel", choices=["replicas", "ulysses"], default="replicas",
+    p.add_argument("--parallel", choices=["replicas", "ulysses", "ring"], default="replicas",
                    help="N > 1: independent replicas per rank (default), or one sequence split "
-                        "over the ranks with Ulysses context parallelism (strong scaling; heads "
-                        "and tokens must divide by N)")
+                        "over the ranks with context parallelism, strong scaling: ulysses (token "
+                        "slices <-> head groups; heads and tokens divide by N) or ring (K/V "
+                        "blocks passed around; tokens divide by N)")
     p.add_argument("--case", choices=["temporal720", "spatial720", "window720", "cross720"],
                    help="run only this secondary kernel (warm-up + --steps launches, one "
                         "JSON line); a small, single-kernel command for profilers")
@@ -538,7 +539,16 @@ def extras(va, device, stream, peak_tf, peak_gbs):
         "scatter_frac_hbm": round(6 * tb / s_ms / 1e6 / peak_gbs, 4),
         "gather_ms": round(g_ms, 4), "gather_gbs": round(2 * tb / g_ms / 1e6, 1),
         "gather_frac_hbm": round(2 * tb / g_ms / 1e6 / peak_gbs, 4)}
-    del q, k, v, ua
+    # the ring step on one rank: key/query load with RoPE, one block product
+    # (the cross-attention form, with LSE) and the fp32 merge
+    from full_spatiotemporal_attention_b200.ring import RingAttention
+    ra = RingAttention(g, w.batch, w.heads, world=1, rank=0, device=device)
+    _, r_ms = timed_loop(ev_pair(lambda: ra(q, k, v)), 5, 3, 1, device)
+    torch.cuda.synchronize()
+    ra.close()
+    out["ring480_1rank"] = {"step_ms": round(r_ms, 4),
+                            "tflops": round(full_flops(w) / r_ms / 1e9, 1)}
+    del q, k, v, ua, ra
     torch.cuda.empty_cache()
     return out
 
@@ -558,6 +568,8 @@ def bench_ulysses(args, rank, world, local):
     torch.cuda.set_device(device)
     w = si.WORKLOADS[args.workload]
     g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    if args.parallel == "ring":
+        return bench_ring(args, rank, world, device, w, g)
     ua = UlyssesAttention(g, w.batch, w.heads, world=world, rank=rank, device=device)
     t0, t1 = ua.plan.token_range
     host = [np.ascontiguousarray(x[:, :, t0:t1]) for x in si.qkv(w)]
@@ -654,6 +666,71 @@ def bench_ulysses(args, rank, world, local):
     }
 
 
+def bench_ring(args, rank, world, device, w, g):
+    """Ring context parallelism: each rank keeps its query slice and sees
+    every rank's K/V block in turn; the step's time is the slowest rank's."""
+    import numpy as np
+    import torch
+    import full_spatiotemporal_attention_b200 as va
+    from full_spatiotemporal_attention_b200.ring import RingAttention
+    import seeded_inputs as si
+    ra = RingAttention(g, w.batch, w.heads, world=world, rank=rank, device=device)
+    nl = w.N // world
+    host = [np.ascontiguousarray(x[:, :, rank * nl:(rank + 1) * nl]) for x in si.qkv(w)]
+    q, k, v = (to_dev(x, device) for x in host)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.5)
+    window = []
+    def step(i):
+        ra(q, k, v)
+    step_ms, _ = timed_loop(step, args.steps, args.warmup, world, device, window=window)
+    clocks = sampler.stop(*window)
+    step_ms = max_over_ranks(step_ms, world, device)
+    qh, kh, vh = (torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in host)
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd = (torch.empty_like(q) for _ in range(3))
+
+    def e2e_step(i):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        oh.copy_(ra(qd, kd, vd), non_blocking=True)
+    e2e_ms, _ = timed_loop(e2e_step, args.e2e_steps, 3, world, device)
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
+    torch.cuda.synchronize()
+    assert va.device_error() == 0, "a peer wait gave up"
+    ra.close(barrier=(lambda: barrier(world)))
+    flops = full_flops(w)
+    peak_tf, _, peak_src = peaks()
+    shard = w.batch * w.heads * nl * HEAD_DIM * 2
+    cfg = job_config(w, world)
+    cfg.update(global_batch=w.batch,
+               parallelism=f"ring x{world} (K/V blocks passed around the ranks over peer memory)")
+    value = flops / (step_ms / 1e3) / 1e12
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded splitmix64 + Box-Muller bf16 N(0,1))", "config": cfg,
+        "pct_of_peak": round(100.0 * value / world / peak_tf, 2),
+        "e2e": {"value": round(flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": 3 * shard,
+                "d2h_bytes_per_step": shard},
+        "gpu_launches": (1 + 3 * world + 4 * (world - 1)) * args.steps,
+        "roofline": {"bound": "tensor", "achieved": round(value / world, 2), "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": round(value / world / peak_tf, 4), "traffic": None,
+                     "kernel": "whole ring step (no separate kernel timing)",
+                     "peak_source": f"{peak_src} bf16 dense (burst)"},
+        "clocks": clocks,
+    }
+
+
 def run_case(args):
     """One secondary kernel alone on the 720p clip, for profiling: `--warmup`
     untimed and `--steps` timed launches.  The temporal pass takes raw keys
@@ -746,7 +823,7 @@ def main():
         print(json.dumps(run_case(args)), flush=True)
         return
     rank, world, local = init_dist("nccl")
-    line = (bench_ulysses if args.parallel == "ulysses" else bench_ours)(args, rank, world, local)
+    line = (bench_ours if args.parallel == "replicas" else bench_ulysses)(args, rank, world, local)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

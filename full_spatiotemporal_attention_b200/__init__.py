@@ -37,7 +37,9 @@ SYMBOLS = ("va3d_status_string", "va3d_version", "va3d_grid_from_video",
            "va3d_cross_workspace_bytes", "attn_cross_fwd", "attn_window_fwd",
            "va3d_watchdog_selftest", "va3d_ulysses_region_bytes", "va3d_ulysses_offsets",
            "va3d_region_alloc", "va3d_region_free", "va3d_ipc_export", "va3d_ipc_open",
-           "va3d_ipc_close", "va3d_ulysses_scatter", "va3d_ulysses_gather", "va3d_ulysses_wait")
+           "va3d_ipc_close", "va3d_ulysses_scatter", "va3d_ulysses_gather", "va3d_ulysses_wait",
+           "va3d_ring_region_bytes", "va3d_ring_offsets", "va3d_ring_load", "va3d_ring_pass",
+           "va3d_ring_free", "va3d_ring_wait", "va3d_ring_merge")
 
 
 class VA3DError(RuntimeError):
@@ -106,6 +108,14 @@ def _load():
     lib.va3d_ulysses_scatter.argtypes = [vp, vp, vp, vpp, i, i, i, i, i, i, gp, u, vp]
     lib.va3d_ulysses_gather.argtypes = [vp, vpp, i, i, i, i, i, i, vp]
     lib.va3d_ulysses_wait.argtypes = [vp, i, ctypes.c_ulonglong, i, i, i, i, i, vp]
+    lib.va3d_ring_region_bytes.argtypes = [i, i, i, i, i]
+    lib.va3d_ring_region_bytes.restype = sz
+    lib.va3d_ring_offsets.argtypes = [i, i, i, i, i, szp, szp, szp, szp]
+    lib.va3d_ring_load.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, gp, u, vp]
+    lib.va3d_ring_pass.argtypes = [vp, vp, i, i, i, i, i, i, vp]
+    lib.va3d_ring_free.argtypes = [vp, vp]
+    lib.va3d_ring_wait.argtypes = [vp, i, ctypes.c_ulonglong, i, i, i, i, i, vp]
+    lib.va3d_ring_merge.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
     return lib
 
 
@@ -438,6 +448,82 @@ def ulysses_wait(region, phase, epoch, world, B, heads, N, device=None):
                                HEAD_DIM, st)
     if rc != VA3D_OK:
         raise VA3DError("va3d_ulysses_wait", rc)
+
+
+# ----------------------------------------------- ring context parallelism
+
+RING_FULL, RING_FREE = 0, 1
+
+
+def ring_region_bytes(B, heads, N, world):
+    return int(lib.va3d_ring_region_bytes(B, heads, N, HEAD_DIM, world))
+
+
+def ring_offsets(B, heads, N, world):
+    """(off_k0, off_v0, off_k1, off_v1) inside a ring region."""
+    offs = [ctypes.c_size_t() for _ in range(4)]
+    rc = lib.va3d_ring_offsets(B, heads, N, HEAD_DIM, world, *(ctypes.byref(o) for o in offs))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ring_offsets", rc)
+    return tuple(int(o.value) for o in offs)
+
+
+def ring_load(q, k, v, q_rot, region, world, rank, grid, *, k_rotated=False):
+    """Turn this rank's slice q, k [B, heads, N/world, 128] at global
+    positions into q_rot and the region's block buffer 0 (with v)."""
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    _check(q_rot, "q_rot", q.shape)
+    B, H, n_loc, D = q.shape
+    rc = lib.va3d_ring_load(_ptr(q), _ptr(k), _ptr(v), _ptr(q_rot), ctypes.c_void_p(region), world,
+                            rank, B, H, n_loc * world, D, ctypes.byref(grid),
+                            VA3D_K_ROTATED if k_rotated else 0, _stream(q))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ring_load", rc)
+
+
+def _cur_stream(device=None):
+    return ctypes.c_void_p(_torch().cuda.current_stream(device).cuda_stream)
+
+
+def ring_pass(region, next_region, buf, world, B, heads, N, device=None):
+    rc = lib.va3d_ring_pass(ctypes.c_void_p(region), ctypes.c_void_p(next_region), buf, world, B,
+                            heads, N, HEAD_DIM, _cur_stream(device))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ring_pass", rc)
+
+
+def ring_free(prev_region, device=None):
+    rc = lib.va3d_ring_free(ctypes.c_void_p(prev_region), _cur_stream(device))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ring_free", rc)
+
+
+def ring_wait(region, counter, count, world, B, heads, N, device=None):
+    rc = lib.va3d_ring_wait(ctypes.c_void_p(region), counter, int(count), world, B, heads, N,
+                            HEAD_DIM, _cur_stream(device))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ring_wait", rc)
+
+
+def ring_merge(o_blk, lse_blk, acc, lse_in, lse_out, *, first, out=None):
+    """Merge a block's (o_blk, lse_blk) into the fp32 accumulator (acc,
+    lse_in) -> (acc, lse_out); with `out`, also write the merged bf16 output."""
+    torch = _torch()
+    _check(o_blk, "o_blk")
+    B, H, n, D = o_blk.shape
+    if acc.dtype != torch.float32 or tuple(acc.shape) != (B, H, n, D) or not acc.is_contiguous():
+        raise ValueError("acc must be a contiguous float32 tensor shaped like o_blk")
+    for t, nm in ((lse_blk, "lse_blk"), (lse_out, "lse_out")) + (() if first else ((lse_in, "lse_in"),)):
+        if t.dtype != torch.float32 or tuple(t.shape) != (B, H, n) or not t.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous float32 [B, heads, n] tensor")
+    if out is not None:
+        _check(out, "out", o_blk.shape)
+    rc = lib.va3d_ring_merge(_ptr(o_blk), _ptr(lse_blk), _ptr(acc), None if first else _ptr(lse_in),
+                             _ptr(lse_out), _ptr(out), B, H, n, 1 if first else 0, _stream(o_blk))
+    if rc != VA3D_OK:
+        raise VA3DError("va3d_ring_merge", rc)
 
 
 class _DeviceMemory:

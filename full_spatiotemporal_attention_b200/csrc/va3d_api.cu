@@ -19,6 +19,7 @@
 #include "attn_temporal.cuh"
 #include "selftest.cuh"
 #include "ulysses.cuh"
+#include "ring.cuh"
 
 using namespace va3d;
 
@@ -161,6 +162,16 @@ int check_ulysses(int B, int heads, int N, int head_dim, int world) {
     if (heads % world != 0 || N % world != 0) return VA3D_ERR_UNSUPPORTED;
     return VA3D_OK;
 }
+
+int check_ring(int B, int heads, int N, int head_dim, int world) {
+    if (world < 1 || world > cp::kMaxWorld) return VA3D_ERR_UNSUPPORTED;
+    int rc;
+    if ((rc = check_sizes(B, heads, N, head_dim)) != VA3D_OK) return rc;
+    if (N % world != 0) return VA3D_ERR_UNSUPPORTED;
+    return VA3D_OK;
+}
+
+bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 
 int check_regions(void *const *regions, int world, int rank) {
     if (regions == nullptr || rank < 0 || rank >= world) return VA3D_ERR_INVALID;
@@ -694,6 +705,122 @@ int va3d_ulysses_wait(const void *region, int phase, unsigned long long epoch, i
     const unsigned long long expected = epoch * static_cast<unsigned long long>(world) * blocks;
     cp::ulysses_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const unsigned long long *>(region), phase, expected);
+    return launch_status();
+}
+
+size_t va3d_ring_region_bytes(int B, int heads, int N, int head_dim, int world) {
+    if (check_ring(B, heads, N, head_dim, world) != VA3D_OK) return 0;
+    return ring::region_layout(B, heads, N, world).bytes;
+}
+
+int va3d_ring_offsets(int B, int heads, int N, int head_dim, int world, size_t *off_k0,
+                      size_t *off_v0, size_t *off_k1, size_t *off_v1) {
+    int rc;
+    if ((rc = check_ring(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
+    if (off_k0 == nullptr || off_v0 == nullptr || off_k1 == nullptr || off_v1 == nullptr)
+        return VA3D_ERR_INVALID;
+    const ring::Layout l = ring::region_layout(B, heads, N, world);
+    *off_k0 = l.k[0];
+    *off_v0 = l.v[0];
+    *off_k1 = l.k[1];
+    *off_v1 = l.v[1];
+    return VA3D_OK;
+}
+
+int va3d_ring_load(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *q_rot,
+                   void *region, int world, int rank, int B, int heads, int N, int head_dim,
+                   const va3d_grid_t *grid, unsigned flags, void *stream) {
+    int rc;
+    if ((rc = check_ring(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
+    if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
+    if (q == nullptr || k == nullptr || v == nullptr || q_rot == nullptr || region == nullptr ||
+        rank < 0 || rank >= world)
+        return VA3D_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_rot) || !aligned256(region))
+        return VA3D_ERR_ALIGNMENT;
+    if (flags & ~static_cast<unsigned>(VA3D_K_ROTATED)) return VA3D_ERR_INVALID;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    const ring::Layout l = ring::region_layout(B, heads, N, world);
+    uint8_t *base = static_cast<uint8_t *>(region);
+    ring::LoadArgs a;
+    a.q = static_cast<const uint4 *>(static_cast<const void *>(q));
+    a.k = static_cast<const uint4 *>(static_cast<const void *>(k));
+    a.v = static_cast<const uint4 *>(static_cast<const void *>(v));
+    a.q_rot = static_cast<uint4 *>(static_cast<void *>(q_rot));
+    a.k0 = reinterpret_cast<uint4 *>(base + l.k[0]);
+    a.v0 = reinterpret_cast<uint4 *>(base + l.v[0]);
+    a.rows = static_cast<long long>(B) * heads;
+    a.n_loc = N / world;
+    a.offset = rank * (N / world);
+    a.rope_q = 1;
+    a.rope_k = (flags & VA3D_K_ROTATED) ? 0 : 1;
+    ring::ring_load_kernel<<<cp::copy_blocks(a.n_loc), cp::kCopyThreads, 0,
+                             static_cast<cudaStream_t>(stream)>>>(a, make_rope_params(grid));
+    return launch_status();
+}
+
+int va3d_ring_pass(const void *region, void *next_region, int buf, int world, int B, int heads,
+                   int N, int head_dim, void *stream) {
+    int rc;
+    if ((rc = check_ring(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
+    if (region == nullptr || next_region == nullptr || (buf != 0 && buf != 1)) return VA3D_ERR_INVALID;
+    if (!aligned256(region) || !aligned256(next_region)) return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    const ring::Layout l = ring::region_layout(B, heads, N, world);
+    const uint8_t *src = static_cast<const uint8_t *>(region);
+    uint8_t *dst = static_cast<uint8_t *>(next_region);
+    const long long rows = static_cast<long long>(B) * heads * (N / world);
+    ring::ring_pass_kernel<<<cp::copy_blocks(rows), cp::kCopyThreads, 0,
+                             static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint4 *>(src + l.k[buf]), reinterpret_cast<const uint4 *>(src + l.v[buf]),
+        reinterpret_cast<uint4 *>(dst + l.k[1 - buf]), reinterpret_cast<uint4 *>(dst + l.v[1 - buf]),
+        rows * 16, dst);
+    return launch_status();
+}
+
+int va3d_ring_free(void *prev_region, void *stream) {
+    int rc;
+    if (prev_region == nullptr) return VA3D_ERR_INVALID;
+    if (!aligned256(prev_region)) return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    ring::ring_free_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint8_t *>(prev_region));
+    return launch_status();
+}
+
+int va3d_ring_wait(const void *region, int counter, unsigned long long count, int world, int B,
+                   int heads, int N, int head_dim, void *stream) {
+    int rc;
+    if ((rc = check_ring(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
+    if (region == nullptr || (counter != ring::kFull && counter != ring::kFree)) return VA3D_ERR_INVALID;
+    if (!aligned256(region)) return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    const long long rows = static_cast<long long>(B) * heads * (N / world);
+    const unsigned long long expected =
+        counter == ring::kFull ? count * static_cast<unsigned long long>(cp::copy_blocks(rows)) : count;
+    cp::ulysses_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const unsigned long long *>(region), counter, expected);
+    return launch_status();
+}
+
+int va3d_ring_merge(const va3d_bf16 *o_blk, const float *lse_blk, float *acc, const float *lse_in,
+                    float *lse_out, va3d_bf16 *out, int B, int heads, int n_rows, int first,
+                    void *stream) {
+    int rc;
+    if ((rc = check_sizes(B, heads, n_rows, kHeadDim)) != VA3D_OK) return rc;
+    if (o_blk == nullptr || lse_blk == nullptr || acc == nullptr || lse_out == nullptr ||
+        (!first && lse_in == nullptr) || (!first && lse_in == lse_out))
+        return VA3D_ERR_INVALID;
+    if (!aligned16(o_blk) || !aligned16(acc) || (out != nullptr && !aligned16(out)) ||
+        (reinterpret_cast<uintptr_t>(lse_blk) & 3u) || (reinterpret_cast<uintptr_t>(lse_out) & 3u) ||
+        (lse_in != nullptr && (reinterpret_cast<uintptr_t>(lse_in) & 3u)))
+        return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    const long long rows = static_cast<long long>(B) * heads * n_rows;
+    ring::ring_merge_kernel<<<cp::copy_blocks(rows), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(static_cast<const void *>(o_blk)), lse_blk,
+        reinterpret_cast<float4 *>(acc), lse_in, lse_out,
+        out ? static_cast<uint4 *>(static_cast<void *>(out)) : nullptr, rows, first ? 1 : 0);
     return launch_status();
 }
 }  // extern "C"

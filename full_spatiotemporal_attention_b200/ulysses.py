@@ -180,6 +180,38 @@ class UlyssesAttention:
                         p.batch, p.heads, p.N, self.device)
         return self.o_shard
 
+    def factorised(self, q, k, v, *, out_spatial=None):
+        """Factorised attention of this rank's slice: (o_spatial, o_temporal),
+        each [B, heads, N/P, 128].  The slice must hold whole frames (P divides
+        T'): the spatial pass then runs on the rank's own frames with no
+        exchange (a frame's t rotation is the same for all its tokens and
+        cancels in q.k, so local frame numbers give the global result), and
+        the temporal pass, which needs every frame of a position, runs on
+        whole sequences of this rank's heads after a Ulysses exchange of the
+        raw keys (its kernel turns only their t range).  o_temporal is a view
+        into the region, valid until the next call."""
+        p, va = self.plan, self.va
+        g = self.grid
+        if g.n_text != 0 or g.T % p.world != 0:
+            raise ValueError(f"factorised slices need whole frames and no text: T'={g.T} "
+                             f"over {p.world} ranks, n_text={g.n_text}")
+        local = va.Grid.make(g.T // p.world, g.H, g.W, 0, (g.d_t, g.d_h, g.d_w), g.theta)
+        out_spatial, _ = va.attn_factorized_fwd(q, k, v, local, temporal=False,
+                                                out_spatial=out_spatial)
+        self.scatter(q, k, v, k_rotated=True)   # raw keys copied as they are
+        va.attn_factorized_fwd(self.qh, self.kh, self.vh, g, spatial=False,
+                               out_temporal=self.o_heads, workspace=self._temporal_workspace())
+        return out_spatial, self.gather()
+
+    def _temporal_workspace(self):
+        if getattr(self, "_tws", None) is None:
+            import torch
+            p = self.plan
+            self._tws = torch.empty(
+                max(self.va.workspace_bytes(p.batch, p.heads_per_rank, p.N, self.grid), 256),
+                dtype=torch.uint8, device=self.device)
+        return self._tws
+
     def __call__(self, q, k, v, *, k_rotated=False):
         """q, k, v: this rank's token slice [B, heads, N/P, 128] bf16; returns
         its slice of the attention output (a view into the region, valid until

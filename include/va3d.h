@@ -374,6 +374,84 @@ int va3d_ulysses_gather(const va3d_bf16 *o_heads, void *const *regions, int worl
 int va3d_ulysses_wait(const void *region, int phase, unsigned long long epoch, int world, int B,
                       int heads, int N, int head_dim, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Ring context parallelism (no head split, so any number of heads).
+ *
+ * Rank r holds tokens [r*N/world, (r+1)*N/world) of every head.
+ * va3d_ring_load turns this rank's q and k by 3D RoPE at their global
+ * positions (positions are absolute: handbook "A video model's
+ * architecture", section "Position: RoPE in three dimensions") into q_rot
+ * and the region's block buffer 0, with v.  Then for steps s = 0..world-1
+ * the rank attends q_rot to the block in buffer s % 2 with attn_cross_fwd
+ * (no RoPE; its LSE kept), merges that partial output into an fp32
+ * accumulator with va3d_ring_merge (log-sum-exp weights), and, except at the
+ * last step, copies the block to the next rank's buffer (s + 1) % 2 with
+ * va3d_ring_pass.  Ordering, all stream-ordered and bounded (2 s, then
+ * VA3D_DEVERR_TIMEOUT_PEER): before va3d_ring_pass of step s of call c,
+ * va3d_ring_wait(free, (c-1)*world + s) (the next rank has finished the
+ * products that read that buffer); after each product va3d_ring_free on the
+ * previous rank's region; before the product of step s+1,
+ * va3d_ring_wait(full, (c-1)*(world-1) + s + 1) (the block has landed).
+ *
+ * Region (one per rank, from va3d_region_alloc; mapped into the previous
+ * rank with the IPC calls): a 256-byte header with two u64 counters (full,
+ * free), then K0, V0, K1, V1, each [B, heads, N/world, 128] bf16.
+ * Requirements: 1 <= world <= 8, N divisible by world, 0 <= rank < world.
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of one rank's ring region; 0 if the sizes are invalid. */
+size_t va3d_ring_region_bytes(int B, int heads, int N, int head_dim, int world);
+
+/* Byte offsets of K0, V0, K1, V1 inside a ring region (256-byte aligned).
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED. */
+int va3d_ring_offsets(int B, int heads, int N, int head_dim, int world, size_t *off_k0,
+                      size_t *off_v0, size_t *off_k1, size_t *off_v1);
+
+/*
+ * q, k, v: this rank's slice [B, heads, N/world, 128] bf16; q_rot: output of
+ * the same shape (device, 16-byte aligned); region: this rank's region.
+ * Keys are copied as they are if flags has VA3D_K_ROTATED.  Text tokens
+ * (global index >= T'H'W') are not turned.  Asynchronous on `stream`.
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _ALIGNMENT, _DEVICE, _CUDA.
+ */
+int va3d_ring_load(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *q_rot,
+                   void *region, int world, int rank, int B, int heads, int N, int head_dim,
+                   const va3d_grid_t *grid, unsigned flags, void *stream);
+
+/*
+ * Copy block buffer `buf` (0 or 1) of this rank's region into buffer 1-buf
+ * of `next_region` (the next rank's region, mapped here), then add one per
+ * block of its grid to the next rank's `full` counter.
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _ALIGNMENT, _DEVICE, _CUDA.
+ */
+int va3d_ring_pass(const void *region, void *next_region, int buf, int world, int B, int heads,
+                   int N, int head_dim, void *stream);
+
+/* Add one to the `free` counter of `prev_region` (the previous rank's).
+ * Errors: VA3D_ERR_INVALID, _ALIGNMENT, _DEVICE, _CUDA. */
+int va3d_ring_free(void *prev_region, void *stream);
+
+/*
+ * Bounded stream-ordered wait on this rank's counter `counter` (0 full,
+ * 1 free): until `count` passes have landed (full; count * the pass grid's
+ * blocks signals) or `count` frees have arrived (free).
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _ALIGNMENT, _DEVICE, _CUDA.
+ */
+int va3d_ring_wait(const void *region, int counter, unsigned long long count, int world, int B,
+                   int heads, int N, int head_dim, void *stream);
+
+/*
+ * Merge one block's output o_blk [B, heads, n_rows, 128] bf16 and its LSE
+ * lse_blk [B, heads, n_rows] fp32 (natural log) into the accumulator acc
+ * [B, heads, n_rows, 128] fp32 whose LSE is lse_in; writes the merged LSE to
+ * lse_out (a different buffer).  first != 0: the accumulator starts as this
+ * block (lse_in unused).  out (nullable): also write the merged output as
+ * bf16.  Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _ALIGNMENT, _DEVICE, _CUDA.
+ */
+int va3d_ring_merge(const va3d_bf16 *o_blk, const float *lse_blk, float *acc, const float *lse_in,
+                    float *lse_out, va3d_bf16 *out, int B, int heads, int n_rows, int first,
+                    void *stream);
+
 #ifdef __cplusplus
 }
 #endif

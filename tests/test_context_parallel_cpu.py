@@ -1,11 +1,11 @@
-"""Host logic of Ulysses context parallelism on the CPU.
+"""Host logic of context parallelism (Ulysses and ring forms) on the CPU.
 
-The exchange itself runs in the library's kernels (tested on a GPU with
-emulated ranks).  Here two gloo ranks run ``UlyssesAttention`` over a fake
-backend that records every call: the IPC handles travel through
-``all_gather_object``, each rank must map exactly its peers' regions in rank
-order, and every call must scatter, wait, attend, gather and wait with the
-right epoch."""
+The exchanges themselves run in the library's kernels (tested on a GPU with
+emulated ranks).  Here ``UlyssesAttention`` and ``RingAttention`` run over a
+fake backend that records every call (two gloo ranks for the Ulysses form):
+the IPC handles travel through ``all_gather_object``, each rank must map
+exactly the regions it needs in rank order, and every call must issue its
+copies, waits, products and merges in order with the right counts."""
 import json
 import os
 import socket
@@ -41,6 +41,8 @@ class FakeBackend:
     PHASE_SCATTER, PHASE_GATHER = 0, 1
 
     def __init__(self, rank):
+        import full_spatiotemporal_attention_b200 as va
+        self.Grid = va.Grid          # a plain ctypes structure, no device involved
         self.rank = rank
         self.calls = []
 
@@ -80,6 +82,12 @@ class FakeBackend:
 
     def ulysses_wait(self, region, phase, epoch, world, B, H, N, device=None):
         self.calls.append(("wait", region, phase, epoch, world))
+
+    def attn_factorized_fwd(self, q, k, v, grid, spatial=True, temporal=True, out_spatial=None,
+                            out_temporal=None, workspace=None):
+        self.calls.append(("factorised", tuple(q.shape), [grid.T, grid.H, grid.W], spatial,
+                           temporal))
+        return out_spatial, out_temporal
 
     def attn3d_full_fwd(self, q, k, v, grid, k_rotated=False, out=None, workspace=None):
         self.calls.append(("attn", tuple(q.shape), k_rotated))
@@ -161,6 +169,36 @@ def test_single_rank_needs_no_exchange():
     ua.close()   # idempotent
 
 
+def test_factorised_call_sequence():
+    """Spatial pass on the rank's own frames (local grid, no exchange), then
+    the raw keys exchanged as they are and the temporal pass on whole
+    sequences of the rank's heads."""
+    import torch
+    from full_spatiotemporal_attention_b200.ulysses import UlyssesAttention
+    import full_spatiotemporal_attention_b200 as va
+    fake = FakeBackend(1)
+    g = va.Grid.make(6, 4, 4)                       # 96 tokens, 2 frames per rank
+    ua = UlyssesAttention(g, 1, 6, world=3, rank=1, device="cpu", backend=fake,
+                          exchange=lambda h: [b"handle-of-0x10000", h, b"handle-of-0x30000"])
+    x = torch.zeros(ua.plan.local_shape, dtype=torch.bfloat16)
+    fake.calls.clear()
+    ua.factorised(x, x, x)
+    regions = [0x10000 + 0x7000000, 0x20000, 0x30000 + 0x7000000]
+    assert [list(c) for c in fake.calls] == [
+        ["factorised", (1, 6, 32, 128), [2, 4, 4], True, False],
+        ["scatter", regions, 1, True],
+        ["wait", 0x20000, 0, 1, 3],
+        ["factorised", (1, 2, 96, 128), [6, 4, 4], False, True],
+        ["gather", regions, 1, 6],
+        ["wait", 0x20000, 1, 1, 3]]
+    # frames that do not split over the ranks, or text tokens
+    ua2 = UlyssesAttention(va.Grid.make(5, 4, 4, n_text=1), 1, 3, world=3, rank=0, device="cpu",
+                           backend=FakeBackend(0), exchange=lambda h: [h, h, h])
+    y = torch.zeros(ua2.plan.local_shape, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="whole frames"):
+        ua2.factorised(y, y, y)
+
+
 def test_failed_exchange_releases_the_region():
     from full_spatiotemporal_attention_b200.ulysses import UlyssesAttention
     import full_spatiotemporal_attention_b200 as va
@@ -169,3 +207,83 @@ def test_failed_exchange_releases_the_region():
         UlyssesAttention(va.Grid.make(2, 4, 4), 1, 2, world=2, rank=1, device="cpu",
                          backend=fake, exchange=lambda h: [h])
     assert fake.calls[-1] == ("free", 0x20000)
+
+
+class FakeRingBackend(FakeBackend):
+    RING_FULL, RING_FREE = 0, 1
+
+    def ring_region_bytes(self, B, H, N, world):
+        return 1 << 20
+
+    def ring_offsets(self, B, H, N, world):
+        return 256, 512, 768, 1024
+
+    def cross_workspace_bytes(self, B, H, Nq, Nkv):
+        return 4096
+
+    def ring_load(self, q, k, v, q_rot, region, world, rank, grid, k_rotated=False):
+        self.calls.append(("load", region, world, rank, k_rotated))
+
+    def ring_wait(self, region, counter, count, world, B, H, N, device=None):
+        self.calls.append(("wait", region, counter, count))
+
+    def ring_pass(self, region, next_region, buf, world, B, H, N, device=None):
+        self.calls.append(("pass", region, next_region, buf))
+
+    def attn_cross_fwd(self, q, k, v, out=None, lse=None, workspace=None):
+        self.calls.append(("product",))
+        return out, lse
+
+    def ring_free(self, prev_region, device=None):
+        self.calls.append(("free_signal", prev_region))
+
+    def ring_merge(self, o_blk, lse_blk, acc, lse_in, lse_out, first, out=None):
+        self.calls.append(("merge", first, out is not None))
+
+
+def test_ring_call_sequence():
+    """Rank 1 of 3: neighbours mapped (next = rank 2, previous = rank 0); per
+    call one load, then per step the free wait and pass (not at the last
+    step), the product, the free signal to the previous rank, the merge (the
+    last one writes the output) and the full wait (not at the last step),
+    with counts that grow across calls."""
+    import torch
+    from full_spatiotemporal_attention_b200.ring import RingAttention
+    import full_spatiotemporal_attention_b200 as va
+    fake = FakeRingBackend(1)
+    handles = [b"handle-of-0x10000", None, b"handle-of-0x30000"]
+    ra = RingAttention(va.Grid.make(3, 4, 4), 1, 2, world=3, rank=1, device="cpu", backend=fake,
+                       exchange=lambda h: [handles[0], h, handles[2]])
+    own, nxt, prv = 0x20000, 0x30000 + 0x7000000, 0x10000 + 0x7000000
+    assert (ra.region, ra.next_region, ra.prev_region) == (own, nxt, prv)
+    x = torch.zeros((1, 2, 16, 128), dtype=torch.bfloat16)
+    for c in (1, 2):
+        fake.calls.clear()
+        assert ra(x, x, x) is ra.out
+        expect = [("load", own, 3, 1, False)]
+        for s in range(3):
+            if s < 2:
+                expect += [("wait", own, 1, (c - 1) * 3 + s), ("pass", own, nxt, s % 2)]
+            expect += [("product",), ("free_signal", prv), ("merge", s == 0, s == 2)]
+            if s < 2:
+                expect += [("wait", own, 0, (c - 1) * 2 + s + 1)]
+        assert fake.calls == expect
+    ra.close()
+    assert fake.calls[-3:] == [("close", nxt), ("close", prv), ("free", own)]
+
+
+def test_ring_two_ranks_share_one_neighbour():
+    """With two ranks the next and the previous rank are the same one: it is
+    mapped once and unmapped once."""
+    from full_spatiotemporal_attention_b200.ring import RingAttention
+    import full_spatiotemporal_attention_b200 as va
+    fake = FakeRingBackend(0)
+    ra = RingAttention(va.Grid.make(2, 4, 4), 1, 1, world=2, rank=0, device="cpu", backend=fake,
+                       exchange=lambda h: [h, b"handle-of-0x20000"])
+    assert ra.next_region == ra.prev_region == 0x20000 + 0x7000000
+    ra.close()
+    assert [c for c in fake.calls if c[0] in ("open", "close")] == [
+        ("open", 0x20000 + 0x7000000), ("close", 0x20000 + 0x7000000)]
+    with pytest.raises(ValueError, match="split"):
+        RingAttention(va.Grid.make(1, 3, 3), 1, 1, world=2, rank=0, device="cpu",
+                      backend=FakeRingBackend(0), exchange=lambda h: [h, h])

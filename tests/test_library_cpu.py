@@ -207,6 +207,35 @@ def test_ulysses_bad_arguments_rejected_before_any_device_call(va):
         va.ipc_open(b"short")
 
 
+def test_ring_region_layout_and_bad_arguments(va):
+    """Ring region = 256-byte header, then K0, V0, K1, V1 of [B, heads, N/P, 128]."""
+    blk = 2 * 12 * (7800 // 8) * 256
+    assert va.ring_offsets(2, 12, 7800, 8) == (256, 256 + blk, 256 + 2 * blk, 256 + 3 * blk)
+    assert va.ring_region_bytes(2, 12, 7800, 8) == 256 + 4 * blk
+    # no head split, so 12 heads over 8 ranks is fine; tokens must split
+    assert va.ring_region_bytes(1, 12, 7801, 8) == 0
+    assert va.ring_region_bytes(1, 12, 7800, 9) == 0
+    lib = va.lib
+    g = va.Grid.make(2, 4, 4)
+    gp = ctypes.byref(g)
+    buf = ctypes.create_string_buffer(4096 + 256)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256)
+    q16 = ctypes.c_void_p(p.value + 16)
+    assert lib.va3d_ring_load(p, p, p, p, p, 2, 2, 1, 2, 32, 128, gp, 0, None) == -1    # rank
+    assert lib.va3d_ring_load(p, p, p, p, p, 3, 0, 1, 2, 32, 128, gp, 0, None) == -2    # 32 % 3
+    assert lib.va3d_ring_load(p, p, p, p, q16, 2, 0, 1, 2, 32, 128, gp, 0, None) == -3  # region
+    assert lib.va3d_ring_load(p, p, p, p, p, 2, 0, 1, 2, 34, 128, gp, 0, None) == -1    # grid
+    assert lib.va3d_ring_pass(p, p, 2, 2, 1, 2, 32, 128, None) == -1                   # buffer
+    assert lib.va3d_ring_pass(p, q16, 0, 2, 1, 2, 32, 128, None) == -3
+    assert lib.va3d_ring_wait(p, 2, 1, 2, 1, 2, 32, 128, None) == -1
+    assert lib.va3d_ring_free(None, None) == -1
+    # merge: a distinct LSE output unless first; alignment
+    assert lib.va3d_ring_merge(p, p, p, p, p, None, 1, 2, 16, 0, None) == -1
+    assert lib.va3d_ring_merge(p, p, p, None, q16, None, 1, 2, 16, 0, None) == -1      # no lse_in
+    assert lib.va3d_ring_merge(ctypes.c_void_p(p.value + 2), p, p, p, ctypes.c_void_p(p.value + 64),
+                               None, 1, 2, 16, 0, None) == -3
+
+
 def test_binding_has_no_cpu_path(va):
     import torch
     g = va.Grid.make(2, 4, 4)
