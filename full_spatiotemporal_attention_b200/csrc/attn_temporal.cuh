@@ -101,9 +101,11 @@ __device__ __forceinline__ float pow2f(int s) {
 
 template <int MAXT>
 struct Cfg {
-    // Up to 12 warps (168 registers each); at T' = 64 shared memory holds 4.
-    static constexpr int kMaxWarps = 12;
-    static constexpr int kSmemBudget = 208 * 1024;
+    // T' <= 32: up to 14 warps (128 registers each, no spills; at T' = 21
+    // their Q, K, V take 226 KB).  T' <= 64: up to 12 warps (168 registers);
+    // at T' = 64 shared memory holds 4.
+    static constexpr int kMaxWarps = MAXT <= 32 ? 14 : 12;
+    static constexpr int kSmemBudget = (MAXT <= 32 ? 226 : 208) * 1024;
 };
 
 // Shared memory per warp: (Q, K, V) with T rows of 256 bytes.
@@ -442,23 +444,24 @@ temporal_kernel(const __grid_constant__ TemporalArgs a) {
             // every lane is done reading these Q rows before O overwrites them
             // (later groups read only higher rows)
             __syncwarp();
-            // ---- O = P V, 64 output columns at a time, staged into the Q rows as bf16
+            // ---- O = P V, 32 output columns at a time (fewer live accumulators, so
+            // more warps fit), staged into the Q rows as bf16
 #pragma unroll
-            for (int dh = 0; dh < 2; ++dh) {
-                float oacc[MG][8][4];
+            for (int dh = 0; dh < 4; ++dh) {
+                float oacc[MG][4][4];
 #pragma unroll
                 for (int m = 0; m < MG; ++m)
 #pragma unroll
-                    for (int nt = 0; nt < 8; ++nt)
+                    for (int nt = 0; nt < 4; ++nt)
                         oacc[m][nt][0] = oacc[m][nt][1] = oacc[m][nt][2] = oacc[m][nt][3] = 0.f;
 #pragma unroll
                 for (int ks = 0; ks < NP; ++ks) {
                     if (ks < n_mt) {
                         const int vrow = min(ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), tl);
 #pragma unroll
-                        for (int dp = 0; dp < 4; ++dp) {
+                        for (int dp = 0; dp < 2; ++dp) {
                             uint32_t b0, b1, b2, b3;
-                            ldsm_x4_t(av + swz(vrow, dh * 8 + dp * 2 + (lane >> 4)), b0, b1, b2, b3);
+                            ldsm_x4_t(av + swz(vrow, dh * 4 + dp * 2 + (lane >> 4)), b0, b1, b2, b3);
 #pragma unroll
                             for (int m = 0; m < MG; ++m) {
                                 mma_bf16(oacc[m][2 * dp], pa[m][ks][0], pa[m][ks][1], pa[m][ks][2],
@@ -473,8 +476,8 @@ temporal_kernel(const __grid_constant__ TemporalArgs a) {
                 for (int m = 0; m < MG; ++m) {
                     const int r0 = (mg + m) * 16 + g, r1 = r0 + 8;
 #pragma unroll
-                    for (int nt = 0; nt < 8; ++nt) {
-                        const int c = dh * 8 + nt;
+                    for (int nt = 0; nt < 4; ++nt) {
+                        const int c = dh * 4 + nt;
                         if (r0 < T)
                             *reinterpret_cast<uint32_t *>(sq + swz(r0, c) + 4 * tq) =
                                 pack_bf16x2(oacc[m][nt][0] * il[m][0], oacc[m][nt][1] * il[m][0]);
