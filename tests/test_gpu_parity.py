@@ -231,7 +231,14 @@ WINDOW_SMALL = [(si.WORKLOADS["tiny"], (1, 2, 4)), (si.WORKLOADS["tiny"], (2, 2,
                 (si.WORKLOADS["tiny"], (1, 1, 1)), (si.WORKLOADS["c17f480"], (5, 6, 4)),
                 (si.WORKLOADS["c17f480"], (1, 10, 26)), (si.WORKLOADS["c17f480"], (5, 15, 13)),
                 (custom("w_odd", 3, 5, 17, heads=3), (3, 5, 1)),
-                (custom("w_b2", 2, 7, 9, batch=2), (2, 7, 3))]
+                (custom("w_b2", 2, 7, 9, batch=2), (2, 7, 3)),
+                # w extents that tile a 128-row tile exactly (8, 16, 32)
+                (custom("w_tma", 3, 6, 32, heads=2), (1, 3, 16)),
+                (custom("w_tma", 3, 6, 32, heads=2), (3, 6, 16)),
+                (custom("w_tma", 3, 6, 32, heads=2), (3, 2, 8)),
+                (custom("w_tma", 3, 6, 32, heads=2), (3, 3, 32)),
+                (custom("w_tma_b2", 2, 4, 16, batch=2), (2, 4, 16)),
+                (custom("w_tma_b2", 2, 4, 16, batch=2), (1, 2, 8))]
 
 
 def window_keys(w, win, n):
@@ -327,6 +334,23 @@ def test_window_gather_matches_the_tma_paths_bit_for_bit(va):
     sp, _ = va.attn_factorized_fwd(q, k, v, g, temporal=False)
     win_sp = va.attn_window_fwd(q, k, v, g, (1, w.H, w.W))
     assert torch.equal(sp.view(torch.int16), win_sp.view(torch.int16))
+
+
+def test_window_rows_of_wide_frames_match_the_tile_paths_bit_for_bit(va):
+    """A 32-wide grid: a window of one frame is the spatial pass and a window
+    of the whole grid full attention, bit for bit."""
+    # frames of 544 tokens (5 key tiles), so that both sides run the same
+    # two-query-tile configuration and split the same tiles
+    w = custom("w_tma_frame", 2, 17, 32, heads=2)
+    q, k, v = (dev(x) for x in si.qkv(w))
+    g = vgrid(va, w)
+    full = va.attn3d_full_fwd(q, k, v, g)
+    win_full = va.attn_window_fwd(q, k, v, g, (w.T, w.H, w.W))
+    assert torch.equal(full.view(torch.int16), win_full.view(torch.int16))
+    sp, _ = va.attn_factorized_fwd(q, k, v, g, temporal=False)
+    win_sp = va.attn_window_fwd(q, k, v, g, (1, w.H, w.W))
+    assert torch.equal(sp.view(torch.int16), win_sp.view(torch.int16))
+    assert va.device_error() == 0
 
 
 def test_window_attention_sampled_rows_full_size(va):
