@@ -722,7 +722,9 @@ def bench_ring(args, rank, world, device, w, g):
         "e2e": {"value": round(flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": 3 * shard,
                 "d2h_bytes_per_step": shard},
-        "gpu_launches": (1 + 3 * world + 4 * (world - 1)) * args.steps,
+        # load; per block: table + product, merge, and (P > 1) the free
+        # signal; per pass: free wait, pass, full wait
+        "gpu_launches": (1 + 3 * world + (world if world > 1 else 0) + 3 * (world - 1)) * args.steps,
         "roofline": {"bound": "tensor", "achieved": round(value / world, 2), "peak": peak_tf,
                      "unit": "TFLOP/s", "frac": round(value / world / peak_tf, 4), "traffic": None,
                      "kernel": "whole ring step (no separate kernel timing)",
