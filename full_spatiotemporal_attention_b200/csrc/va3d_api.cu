@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdint>
@@ -27,6 +28,15 @@ namespace {
 
 constexpr int kHeadDim = 128;
 constexpr double kLog2e = 1.4426950408889634;
+
+// Host-side NVTX range over one entry point (header-only NVTX v3: without a
+// profiler attached the calls return at once and nothing is linked).
+struct TraceRange {
+    explicit TraceRange(const char *name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange &) = delete;
+    TraceRange &operator=(const TraceRange &) = delete;
+};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -447,6 +457,7 @@ size_t va3d_workspace_bytes(int B, int heads, int N, int head_dim, const va3d_gr
 
 int rope3d_apply(const va3d_bf16 *x, va3d_bf16 *y, int B, int heads, int N, int head_dim,
                  const va3d_grid_t *grid, void *stream) {
+    TraceRange trace("va3d.rope3d_apply");
     int rc;
     if ((rc = check_sizes(B, heads, N, head_dim)) != VA3D_OK) return rc;
     if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
@@ -460,6 +471,7 @@ int attn3d_full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, 
                     float *lse, int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
                     float softmax_scale, unsigned flags, void *workspace, size_t workspace_bytes,
                     void *stream) {
+    TraceRange trace("va3d.attn3d_full_fwd");
     if (o == nullptr) return VA3D_ERR_INVALID;
     if (!aligned16(o) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return VA3D_ERR_ALIGNMENT;
@@ -476,6 +488,7 @@ int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 
                         va3d_bf16 *o_spatial, va3d_bf16 *o_temporal, int B, int heads, int N,
                         int head_dim, const va3d_grid_t *grid, float softmax_scale, unsigned flags,
                         void *workspace, size_t workspace_bytes, void *stream) {
+    TraceRange trace("va3d.attn_factorized_fwd");
     if (o_spatial == nullptr && o_temporal == nullptr) return VA3D_ERR_INVALID;
     if ((o_spatial && !aligned16(o_spatial)) || (o_temporal && !aligned16(o_temporal)))
         return VA3D_ERR_ALIGNMENT;
@@ -507,6 +520,7 @@ size_t va3d_cross_workspace_bytes(int B, int heads, int Nq, int Nkv, int head_di
 int attn_cross_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *o,
                    float *lse, int B, int heads, int Nq, int Nkv, int head_dim, float softmax_scale,
                    void *workspace, size_t workspace_bytes, void *stream) {
+    TraceRange trace("va3d.attn_cross_fwd");
     int rc;
     if ((rc = check_sizes(B, heads, Nq, head_dim)) != VA3D_OK) return rc;
     if ((rc = check_sizes(B, heads, Nkv, head_dim)) != VA3D_OK) return rc;
@@ -534,6 +548,7 @@ int attn_window_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, 
                     float *lse, int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
                     int win_t, int win_h, int win_w, float softmax_scale, unsigned flags,
                     void *workspace, size_t workspace_bytes, void *stream) {
+    TraceRange trace("va3d.attn_window_fwd");
     if (o == nullptr || grid == nullptr) return VA3D_ERR_INVALID;
     if (!aligned16(o) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return VA3D_ERR_ALIGNMENT;
@@ -636,6 +651,7 @@ int va3d_ipc_close(void *ptr) {
 int va3d_ulysses_scatter(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
                          void *const *regions, int world, int rank, int B, int heads, int N,
                          int head_dim, const va3d_grid_t *grid, unsigned flags, void *stream) {
+    TraceRange trace("va3d.va3d_ulysses_scatter");
     int rc;
     if ((rc = check_ulysses(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
     if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
@@ -670,6 +686,7 @@ int va3d_ulysses_scatter(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16
 
 int va3d_ulysses_gather(const va3d_bf16 *o_heads, void *const *regions, int world, int rank,
                         int B, int heads, int N, int head_dim, void *stream) {
+    TraceRange trace("va3d.va3d_ulysses_gather");
     int rc;
     if ((rc = check_ulysses(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
     if ((rc = check_regions(regions, world, rank)) != VA3D_OK) return rc;
@@ -695,6 +712,7 @@ int va3d_ulysses_gather(const va3d_bf16 *o_heads, void *const *regions, int worl
 
 int va3d_ulysses_wait(const void *region, int phase, unsigned long long epoch, int world, int B,
                       int heads, int N, int head_dim, void *stream) {
+    TraceRange trace("va3d.va3d_ulysses_wait");
     int rc;
     if ((rc = check_ulysses(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
     if (region == nullptr || (phase != cp::kScatter && phase != cp::kGather) || epoch == 0)
@@ -730,6 +748,7 @@ int va3d_ring_offsets(int B, int heads, int N, int head_dim, int world, size_t *
 int va3d_ring_load(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *q_rot,
                    void *region, int world, int rank, int B, int heads, int N, int head_dim,
                    const va3d_grid_t *grid, unsigned flags, void *stream) {
+    TraceRange trace("va3d.va3d_ring_load");
     int rc;
     if ((rc = check_ring(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
     if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
@@ -761,6 +780,7 @@ int va3d_ring_load(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, v
 
 int va3d_ring_pass(const void *region, void *next_region, int buf, int world, int B, int heads,
                    int N, int head_dim, void *stream) {
+    TraceRange trace("va3d.va3d_ring_pass");
     int rc;
     if ((rc = check_ring(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
     if (region == nullptr || next_region == nullptr || (buf != 0 && buf != 1)) return VA3D_ERR_INVALID;
@@ -779,6 +799,7 @@ int va3d_ring_pass(const void *region, void *next_region, int buf, int world, in
 }
 
 int va3d_ring_free(void *prev_region, void *stream) {
+    TraceRange trace("va3d.va3d_ring_free");
     int rc;
     if (prev_region == nullptr) return VA3D_ERR_INVALID;
     if (!aligned256(prev_region)) return VA3D_ERR_ALIGNMENT;
@@ -790,6 +811,7 @@ int va3d_ring_free(void *prev_region, void *stream) {
 
 int va3d_ring_wait(const void *region, int counter, unsigned long long count, int world, int B,
                    int heads, int N, int head_dim, void *stream) {
+    TraceRange trace("va3d.va3d_ring_wait");
     int rc;
     if ((rc = check_ring(B, heads, N, head_dim, world)) != VA3D_OK) return rc;
     if (region == nullptr || (counter != ring::kFull && counter != ring::kFree)) return VA3D_ERR_INVALID;
@@ -806,6 +828,7 @@ int va3d_ring_wait(const void *region, int counter, unsigned long long count, in
 int va3d_ring_merge(const va3d_bf16 *o_blk, const float *lse_blk, float *acc, const float *lse_in,
                     float *lse_out, va3d_bf16 *out, int B, int heads, int n_rows, int first,
                     void *stream) {
+    TraceRange trace("va3d.va3d_ring_merge");
     int rc;
     if ((rc = check_sizes(B, heads, n_rows, kHeadDim)) != VA3D_OK) return rc;
     if (o_blk == nullptr || lse_blk == nullptr || acc == nullptr || lse_out == nullptr ||
