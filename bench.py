@@ -276,6 +276,70 @@ def timed_loop(fn, steps, warmup, world, device, window=None):
     return total / steps, (sum(inner_ms) / len(inner_ms) if inner_ms else None)
 
 
+def e2e_pipelined(va, g, w, host_bits, steps, world, device, warmup=3):
+    """Per-step time of the end-to-end loop through the public API: each step
+    copies its Q, K, V from pinned host memory (H2D), runs attn3d_full_fwd
+    (key pre-pass, table, attention) and reads its O back (D2H).  Device
+    buffers are double-buffered and the copies run on their own streams, so
+    step i+1's upload and step i-1's download overlap step i's kernels, as a
+    serving loop streams requests; the timed region starts before the first
+    upload and ends after the last download."""
+    import torch
+    comp = torch.cuda.current_stream(device)
+    up = torch.cuda.Stream(device)
+    down = torch.cuda.Stream(device)
+    qh, kh, vh = (torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in host_bits)
+    dev_in = [[torch.empty(qh.shape, dtype=torch.bfloat16, device=device) for _ in range(3)]
+              for _ in range(2)]
+    dev_out = [torch.empty(qh.shape, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    host_out = [torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    ws = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g), dtype=torch.uint8, device=device)
+    ev = lambda: torch.cuda.Event()
+    uploaded, computed, downloaded = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def upload(i):
+        b = i % 2
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(computed[b])          # step i-2 has read these buffers
+            for d, h in zip(dev_in[b], (qh, kh, vh)):
+                d.copy_(h, non_blocking=True)
+            uploaded[b].record(up)
+
+    def run(n, start=None):
+        if start is not None:
+            up.wait_event(start)
+        upload(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                upload(i + 1)
+            comp.wait_event(uploaded[b])
+            if i >= 2:
+                comp.wait_event(downloaded[b])      # step i-2's O has left this buffer
+            q, k, v = dev_in[b]
+            va.attn3d_full_fwd(q, k, v, g, out=dev_out[b], workspace=ws)
+            computed[b].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                host_out[b].copy_(dev_out[b], non_blocking=True)
+                downloaded[b].record(down)
+        comp.wait_stream(down)
+        comp.wait_stream(up)
+
+    run(warmup)
+    torch.cuda.synchronize()
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    run(steps, start=a)
+    b.record(comp)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(a.elapsed_time(b) / steps, world, device)
+
+
 def bench_ours(args, rank, world, local):
     import torch
     import full_spatiotemporal_attention_b200 as va
@@ -335,20 +399,7 @@ def bench_ours(args, rank, world, local):
 
     # end to end through the public API with host buffers
     tensor_bytes = w.batch * w.heads * w.N * HEAD_DIM * 2
-    qh, kh, vh = (torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in (qb, kb, vb))
-    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
-    qd, kd, vd = (torch.empty_like(q) for _ in range(3))
-    ws_full = torch.empty(va.workspace_bytes(w.batch, w.heads, w.N, g), dtype=torch.uint8,
-                          device=device)
-
-    def e2e_step(i):
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        va.attn3d_full_fwd(qd, kd, vd, g, out=o, workspace=ws_full)
-        oh.copy_(o, non_blocking=True)
-    e2e_ms, _ = timed_loop(e2e_step, args.e2e_steps, 3, world, device)
-    e2e_ms = max_over_ranks(e2e_ms, world, device)
+    e2e_ms = e2e_pipelined(va, g, w, (qb, kb, vb), args.e2e_steps, world, device)
 
     line = {
         "metric": METRIC,
@@ -367,7 +418,9 @@ def bench_ours(args, rank, world, local):
         "pct_of_peak": round(100.0 * value / world / peak_tf, 2),
         "e2e": {"value": round(job_tflops(flops, world, e2e_ms), 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4),
-                "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes},
+                "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes,
+                "pipelined": "double-buffered: step i+1's H2D and step i-1's D2H overlap "
+                             "step i's kernels; every step's own copies are in the timed region"},
         "gpu_launches": 3 * args.steps,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf,
                      "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
