@@ -276,6 +276,28 @@ def test_rope_T1_reduces_to_2d_and_HW1_to_1d():
     assert np.abs(y[..., :44] - bf16_bits_to_f64(x)[..., :44]).max() > 1e-3
 
 
+@pytest.mark.parametrize("dims", [(44, 42, 42), (16, 56, 56)])
+def test_temporal_pass_needs_only_the_time_range_turned(dims):
+    """Within one (h, w) position the h and w rotations of a query and a key
+    are the same orthogonal map and cancel in their dot product, so the
+    temporal pass's scores equal those of queries and keys turned by t only
+    (the same tokens on a T' x 1 x 1 grid), with the other dims untouched."""
+    T, H, W = 5, 3, 4
+    g = Grid(T, H, W, dims=dims)
+    x = _rand_bits((2, g.N, 128), 17)
+    rot = oracle.rope3d(x, g)
+    g_t = Grid(T, 1, 1, dims=dims)
+    rng = np.random.default_rng(3)
+    for _ in range(10):
+        h, w = int(rng.integers(0, H)), int(rng.integers(0, W))
+        idx = np.array([(t * H + h) * W + w for t in range(T)])
+        only_t = oracle.rope3d(x[:, idx], g_t)          # token t of the column at (t, 0, 0)
+        np.testing.assert_array_equal(only_t[..., dims[0]:], bf16_bits_to_f64(x[:, idx])[..., dims[0]:])
+        full_scores = rot[0, idx] @ rot[1, idx].T
+        t_scores = only_t[0] @ only_t[1].T
+        np.testing.assert_allclose(full_scores, t_scores, atol=1e-9, rtol=1e-9)
+
+
 def test_rope_pairs_are_adjacent():
     """A unit vector in dim o+2j of a range only mixes with dim o+2j+1."""
     g = Grid(3, 3, 3, dims=(44, 42, 42))
