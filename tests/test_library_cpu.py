@@ -152,6 +152,28 @@ def test_bad_arguments_rejected_before_any_device_call(va):
     assert lib.rope3d_apply(p, p, 1, 2, 32, 128, ctypes.byref(godd), None) == -1
 
 
+def test_empty_inputs_are_rejected(va):
+    """No tokens, no heads or no batch: every entry point returns
+    VA3D_ERR_INVALID before touching a device (there is nothing to compute,
+    and a zero-sized launch would be an error)."""
+    lib = va.lib
+    buf = ctypes.create_string_buffer(4096 + 256)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256)
+    g0 = va.Grid.make(0, 4, 4)
+    g = va.Grid.make(2, 4, 4)
+    for B, H, N, grid in ((1, 2, 0, g0), (1, 0, 32, g), (0, 2, 32, g)):
+        gp = ctypes.byref(grid)
+        assert lib.attn3d_full_fwd(p, p, p, p, None, B, H, N, 128, gp, 0.0, 0, p, 4096, None) == -1
+        assert lib.attn_factorized_fwd(p, p, p, p, p, B, H, N, 128, gp, 0.0, 0, p, 4096, None) == -1
+        assert lib.attn_window_fwd(p, p, p, p, None, B, H, N, 128, gp, 1, 2, 2, 0.0, 0, p, 4096,
+                                   None) == -1
+        assert lib.rope3d_apply(p, p, B, H, N, 128, gp, None) == -1
+        assert lib.va3d_workspace_bytes(B, H, N, 128, gp, 0) == 0
+    assert lib.attn_cross_fwd(p, p, p, p, None, 1, 2, 0, 8, 128, 0.0, None, 0, None) == -1
+    assert lib.attn_cross_fwd(p, p, p, p, None, 1, 2, 32, 0, 128, 0.0, None, 0, None) == -1
+    assert lib.va3d_grid_from_video(0, 480, 832, 44, 42, 42, 0, ctypes.byref(va.Grid())) == -1
+
+
 def test_ulysses_region_layout(va):
     """Region = 256-byte header, Qh, Kh, Vh [B, heads/P, N, 128] and the O
     shard [B, heads, N/P, 128], bf16 rows of 256 bytes."""
