@@ -20,7 +20,10 @@
  *  - text cross-attention: the same page, section 3.1 (Wan's block);
  *  - local 3D-window attention: anthology-of-the-sota record sota-390
  *    (W.A.L.T's local 3D-window blocks, the one numbered comparison against
- *    full attention it cites).
+ *    full attention it cites);
+ *  - context parallelism (Ulysses and ring exchanges, one process per GPU):
+ *    the same record (long videos turn to context parallelism) and the
+ *    handbook's RoPE section (each rank's token coordinates are absolute).
  *
  * Conventions shared by every entry point
  *  - Tensors are contiguous bf16 (bit patterns, va3d_bf16) of shape
@@ -33,9 +36,10 @@
  *  - RoPE: the head dim is split into ranges [0, d_t), [d_t, d_t+d_h),
  *    [d_t+d_h, 128) turned by t, h and w; inside a range of width d the
  *    adjacent pair (2j, 2j+1) turns by pos * theta^(-2j/d).
- *  - Memory is owned by the caller.  No entry point allocates device memory;
- *    scratch space is the caller's `workspace` (size from
- *    va3d_workspace_bytes).  Device pointers must belong to the current
+ *  - Memory is owned by the caller.  No compute entry point allocates device
+ *    memory; scratch space is the caller's `workspace` (size from
+ *    va3d_workspace_bytes).  The one allocating call, va3d_region_alloc, is a
+ *    set-up call for the context-parallel exchange regions.  Device pointers must belong to the current
  *    device.  Two calls that share a workspace must not overlap in time.
  *  - Calls are asynchronous on `stream` (NULL = legacy default stream).  The
  *    return value reports argument errors and launch errors only; device-side
