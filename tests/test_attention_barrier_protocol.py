@@ -203,3 +203,61 @@ def test_late_v_release_with_one_stage_and_gathered_rows_deadlocks(n_kv):
             stuck = True
             break
     assert stuck
+
+
+# --------------------------------------------------- split-tile epilogue
+
+def _split_units(order_seed):
+    """The two units of a split tile (each over half of the keys): every
+    softmax thread stores its normalised partial row and (max, sum) to the
+    scratch and fences; once the whole CTA has (B_EPI), one thread adds 1 to
+    the tile's counter (cleared by the table kernel before the launch) and
+    publishes the old value (B_EPI_GO); the unit that saw 1 merges both
+    halves.  Each unit is a list of events over a shared state; the rows of
+    a unit are modelled as two threads to let their stores interleave."""
+    state = {"count": 0, "written": [[False, False], [False, False]], "merged_by": [],
+             "seen": [None, None]}
+
+    def unit(u):
+        ev = []
+        for row in range(2):
+            ev.append(lambda st, row=row: st["written"][u].__setitem__(row, True))
+        # B_EPI: all rows stored and fenced before the counting thread runs
+        ev.append(("epi", u))
+        def count(st):
+            st["seen"][u] = st["count"]
+            st["count"] += 1
+        ev.append(count)
+        def merge(st):
+            if st["seen"][u] == 1:
+                other = 1 - u
+                assert all(st["written"][other]), "merged a half that was not fully stored"
+                assert all(st["written"][u])
+                st["merged_by"].append(u)
+        ev.append(merge)
+        return ev
+    return state, [unit(0), unit(1)]
+
+
+def test_split_tile_is_merged_once_and_only_when_complete():
+    for seed in range(500):
+        rng = random.Random(seed)
+        state, units = _split_units(seed)
+        pcs = [0, 0]
+        while pcs != [len(units[0]), len(units[1])]:
+            ready = []
+            for u in (0, 1):
+                if pcs[u] >= len(units[u]):
+                    continue
+                ev = units[u][pcs[u]]
+                if isinstance(ev, tuple) and ev[0] == "epi" and not all(state["written"][u]):
+                    continue
+                ready.append(u)
+            u = rng.choice(ready)
+            ev = units[u][pcs[u]]
+            if not isinstance(ev, tuple):
+                ev(state)
+            pcs[u] += 1
+        assert state["count"] == 2
+        assert len(state["merged_by"]) == 1
+        assert sorted(state["seen"]) == [0, 1]
