@@ -5,7 +5,8 @@
 //
 // The pass is HBM-bound (each position reads T' rows of Q, K, V and writes T'
 // rows of O; its 4*T'^2*d FLOPs are small), so the design goal is streaming:
-//  - persistent warps (up to 12 per block, as many as shared memory holds), one
+//  - persistent warps (up to 14 per block for T' <= 32, 12 for T' <= 64; as
+//    many as shared memory holds), one
 //    (batch*head, position) task at a time, rows fetched with 16-byte
 //    cp.async (each row is 256 contiguous bytes); the other resident warps
 //    compute while one waits for its rows;
