@@ -73,10 +73,14 @@ class Grid(ctypes.Structure):
 
 
 def _load():
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(
-            f"{LIB_PATH} is not built; run `python -m full_spatiotemporal_attention_b200.build` "
-            "or __graft_entry__.build() (nvcc with sm_100a)")
+    # Build (or rebuild, when the sources changed) with nvcc first; without
+    # nvcc and without a library built from these sources the import fails.
+    from . import build as _build
+    try:
+        _build.build()
+    except (OSError, RuntimeError) as e:
+        raise ImportError(f"{LIB_PATH} could not be built from the current sources "
+                          f"(nvcc for sm_100a): {e}") from e
     lib = ctypes.CDLL(LIB_PATH)
     vp, i, u, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t, ctypes.c_float
     gp = ctypes.POINTER(Grid)
@@ -177,11 +181,63 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
+def _run(name, device, *args):
+    """Call C entry point `name` with `device` current (the library launches on
+    the current device and takes its per-device state from it), raising
+    VA3DError on a non-zero status."""
+    with _torch().cuda.device(device):
+        rc = getattr(lib, name)(*args)
+    if rc != VA3D_OK:
+        raise VA3DError(name, rc)
+
+
+def _check_lse(lse, shape):
+    torch = _torch()
+    if lse is not None and (not isinstance(lse, torch.Tensor) or lse.dtype != torch.float32
+                            or tuple(lse.shape) != tuple(shape) or not lse.is_contiguous()
+                            or not lse.is_cuda):
+        raise ValueError(f"lse must be a contiguous CUDA float32 {list(shape)} tensor")
+    return lse
+
+
+def _device(device=None):
+    """`device` as a torch.device (the current CUDA device when None)."""
+    torch = _torch()
+    return torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+
+
+def _cur_stream(device=None):
+    return ctypes.c_void_p(_torch().cuda.current_stream(device).cuda_stream)
+
+
+def _same_device(ref, *ts):
+    for t in ts:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"tensors must be on one device: {t.device} != {ref.device}")
+
+
+# Workspaces the binding keeps for calls that pass none, one per (device,
+# stream), grown on demand: calls on one stream are ordered, so they can share
+# one buffer, and calls on different streams never do.
+_WORKSPACES = {}
+
+
+def release_workspaces():
+    """Drop the workspaces kept for calls that passed none (synchronise first
+    if calls that use them may still be running)."""
+    _WORKSPACES.clear()
+
+
 def _workspace(q, grid, k_rotated, workspace):
     B, H, N, _ = q.shape
     need = workspace_bytes(B, H, N, grid, k_rotated)
     if workspace is None:
-        workspace = _torch().empty(max(need, 256), dtype=_torch().uint8, device=q.device)
+        torch = _torch()
+        key = (q.device.index, torch.cuda.current_stream(q.device).cuda_stream)
+        workspace = _WORKSPACES.get(key)
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+            _WORKSPACES[key] = workspace
     if workspace.numel() * workspace.element_size() < need:
         raise ValueError(f"workspace holds {workspace.numel()} bytes, needs {need}")
     return workspace
@@ -193,10 +249,9 @@ def rope3d_apply(x, grid, out=None):
     if out is None:
         out = _torch().empty_like(x)
     _check(out, "out", x.shape)
+    _same_device(x, out)
     B, H, N, D = x.shape
-    rc = lib.rope3d_apply(_ptr(x), _ptr(out), B, H, N, D, ctypes.byref(grid), _stream(x))
-    if rc != VA3D_OK:
-        raise VA3DError("rope3d_apply", rc)
+    _run("rope3d_apply", x.device, _ptr(x), _ptr(out), B, H, N, D, ctypes.byref(grid), _stream(x))
     return out
 
 
@@ -215,16 +270,12 @@ def attn3d_full_fwd(q, k, v, grid, *, scale=None, return_lse=False, k_rotated=Fa
     _check(out, "out", q.shape)
     if return_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N)
-                            or not lse.is_contiguous() or not lse.is_cuda):
-        raise ValueError("lse must be a contiguous CUDA float32 [B, heads, N] tensor")
+    _check_lse(lse, (B, H, N))
     ws = _workspace(q, grid, k_rotated, workspace)
-    rc = lib.attn3d_full_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
-                             ctypes.byref(grid), float(scale or 0.0),
-                             VA3D_K_ROTATED if k_rotated else 0, _ptr(ws),
-                             ws.numel() * ws.element_size(), _stream(q))
-    if rc != VA3D_OK:
-        raise VA3DError("attn3d_full_fwd", rc)
+    _same_device(q, k, v, out, lse, ws)
+    _run("attn3d_full_fwd", q.device, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
+         ctypes.byref(grid), float(scale or 0.0), VA3D_K_ROTATED if k_rotated else 0, _ptr(ws),
+         ws.numel() * ws.element_size(), _stream(q))
     return (out, lse) if (return_lse or lse is not None) else out
 
 
@@ -243,11 +294,11 @@ def attn3d_full_fwd_noalloc(q, k, v, grid, *, scale=None, return_lse=False, k_ro
     _check(out, "out", q.shape)
     if return_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    rc = lib.attn3d_full_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
-                                     ctypes.byref(grid), float(scale or 0.0),
-                                     VA3D_K_ROTATED if k_rotated else 0, _stream(q))
-    if rc != VA3D_OK:
-        raise VA3DError("attn3d_full_fwd_noalloc", rc)
+    _check_lse(lse, (B, H, N))
+    _same_device(q, k, v, out, lse)
+    _run("attn3d_full_fwd_noalloc", q.device, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+         B, H, N, D, ctypes.byref(grid), float(scale or 0.0), VA3D_K_ROTATED if k_rotated else 0,
+         _stream(q))
     return (out, lse) if (return_lse or lse is not None) else out
 
 
@@ -271,12 +322,10 @@ def attn_factorized_fwd(q, k, v, grid, *, spatial=True, temporal=True, scale=Non
         if t is not None:
             _check(t, nm, q.shape)
     ws = _workspace(q, grid, k_rotated, workspace)
-    rc = lib.attn_factorized_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out_spatial),
-                                 _ptr(out_temporal), B, H, N, D, ctypes.byref(grid),
-                                 float(scale or 0.0), VA3D_K_ROTATED if k_rotated else 0,
-                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(q))
-    if rc != VA3D_OK:
-        raise VA3DError("attn_factorized_fwd", rc)
+    _same_device(q, k, v, out_spatial, out_temporal, ws)
+    _run("attn_factorized_fwd", q.device, _ptr(q), _ptr(k), _ptr(v), _ptr(out_spatial),
+         _ptr(out_temporal), B, H, N, D, ctypes.byref(grid), float(scale or 0.0),
+         VA3D_K_ROTATED if k_rotated else 0, _ptr(ws), ws.numel() * ws.element_size(), _stream(q))
     return out_spatial, out_temporal
 
 
@@ -295,17 +344,13 @@ def attn_window_fwd(q, k, v, grid, window, *, scale=None, return_lse=False, k_ro
     _check(out, "out", q.shape)
     if return_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N)
-                            or not lse.is_contiguous() or not lse.is_cuda):
-        raise ValueError("lse must be a contiguous CUDA float32 [B, heads, N] tensor")
+    _check_lse(lse, (B, H, N))
     ws = _workspace(q, grid, k_rotated, workspace)
+    _same_device(q, k, v, out, lse, ws)
     wt, wh, ww = (int(x) for x in window)
-    rc = lib.attn_window_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
-                             ctypes.byref(grid), wt, wh, ww, float(scale or 0.0),
-                             VA3D_K_ROTATED if k_rotated else 0, _ptr(ws),
-                             ws.numel() * ws.element_size(), _stream(q))
-    if rc != VA3D_OK:
-        raise VA3DError("attn_window_fwd", rc)
+    _run("attn_window_fwd", q.device, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
+         ctypes.byref(grid), wt, wh, ww, float(scale or 0.0), VA3D_K_ROTATED if k_rotated else 0,
+         _ptr(ws), ws.numel() * ws.element_size(), _stream(q))
     return (out, lse) if (return_lse or lse is not None) else out
 
 
@@ -331,17 +376,12 @@ def attn_cross_fwd(q, k, v, *, scale=None, return_lse=False, out=None, lse=None,
     _check(out, "out", q.shape)
     if return_lse and lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq)
-                            or not lse.is_contiguous() or not lse.is_cuda):
-        raise ValueError("lse must be a contiguous CUDA float32 [B, heads, Nq] tensor")
-    if workspace is None:
-        workspace = torch.empty(max(cross_workspace_bytes(B, H, Nq, Nkv), 256),
-                                dtype=torch.uint8, device=q.device)
-    rc = lib.attn_cross_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Nq, Nkv, D,
-                            float(scale or 0.0), _ptr(workspace),
-                            workspace.numel() * workspace.element_size(), _stream(q))
-    if rc != VA3D_OK:
-        raise VA3DError("attn_cross_fwd", rc)
+    _check_lse(lse, (B, H, Nq))
+    _same_device(q, k, v, out, lse, workspace)
+    # the workspace is optional here (it only lets the last partial wave split)
+    _run("attn_cross_fwd", q.device, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Nq,
+         Nkv, D, float(scale or 0.0), _ptr(workspace),
+         workspace.numel() * workspace.element_size() if workspace is not None else 0, _stream(q))
     return (out, lse) if (return_lse or lse is not None) else out
 
 
@@ -419,11 +459,10 @@ def ulysses_scatter(q, k, v, regions, rank, grid, *, k_rotated=False):
     _check(v, "v", q.shape)
     B, H, n_loc, D = q.shape
     world = len(regions)
-    rc = lib.va3d_ulysses_scatter(_ptr(q), _ptr(k), _ptr(v), _ptr_array(regions), world, rank, B, H,
-                                  n_loc * world, D, ctypes.byref(grid),
-                                  VA3D_K_ROTATED if k_rotated else 0, _stream(q))
-    if rc != VA3D_OK:
-        raise VA3DError("va3d_ulysses_scatter", rc)
+    _same_device(q, k, v)
+    _run("va3d_ulysses_scatter", q.device, _ptr(q), _ptr(k), _ptr(v), _ptr_array(regions), world,
+         rank, B, H, n_loc * world, D, ctypes.byref(grid), VA3D_K_ROTATED if k_rotated else 0,
+         _stream(q))
 
 
 def ulysses_gather(o_heads, regions, rank, heads):
@@ -434,20 +473,14 @@ def ulysses_gather(o_heads, regions, rank, heads):
     world = len(regions)
     if hpw * world != heads:
         raise ValueError(f"o_heads holds {hpw} heads, expected {heads} / {world}")
-    rc = lib.va3d_ulysses_gather(_ptr(o_heads), _ptr_array(regions), world, rank, B, heads, N, D,
-                                 _stream(o_heads))
-    if rc != VA3D_OK:
-        raise VA3DError("va3d_ulysses_gather", rc)
+    _run("va3d_ulysses_gather", o_heads.device, _ptr(o_heads), _ptr_array(regions), world, rank, B,
+         heads, N, D, _stream(o_heads))
 
 
 def ulysses_wait(region, phase, epoch, world, B, heads, N, device=None):
     """Stream-ordered, bounded wait for every peer's signals of call `epoch`."""
-    torch = _torch()
-    st = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
-    rc = lib.va3d_ulysses_wait(ctypes.c_void_p(region), phase, int(epoch), world, B, heads, N,
-                               HEAD_DIM, st)
-    if rc != VA3D_OK:
-        raise VA3DError("va3d_ulysses_wait", rc)
+    _run("va3d_ulysses_wait", _device(device), ctypes.c_void_p(region), phase, int(epoch), world, B,
+         heads, N, HEAD_DIM, _cur_stream(device))
 
 
 # ----------------------------------------------- ring context parallelism
@@ -476,35 +509,24 @@ def ring_load(q, k, v, q_rot, region, world, rank, grid, *, k_rotated=False):
     _check(v, "v", q.shape)
     _check(q_rot, "q_rot", q.shape)
     B, H, n_loc, D = q.shape
-    rc = lib.va3d_ring_load(_ptr(q), _ptr(k), _ptr(v), _ptr(q_rot), ctypes.c_void_p(region), world,
-                            rank, B, H, n_loc * world, D, ctypes.byref(grid),
-                            VA3D_K_ROTATED if k_rotated else 0, _stream(q))
-    if rc != VA3D_OK:
-        raise VA3DError("va3d_ring_load", rc)
-
-
-def _cur_stream(device=None):
-    return ctypes.c_void_p(_torch().cuda.current_stream(device).cuda_stream)
+    _same_device(q, k, v, q_rot)
+    _run("va3d_ring_load", q.device, _ptr(q), _ptr(k), _ptr(v), _ptr(q_rot), ctypes.c_void_p(region),
+         world, rank, B, H, n_loc * world, D, ctypes.byref(grid),
+         VA3D_K_ROTATED if k_rotated else 0, _stream(q))
 
 
 def ring_pass(region, next_region, buf, world, B, heads, N, device=None):
-    rc = lib.va3d_ring_pass(ctypes.c_void_p(region), ctypes.c_void_p(next_region), buf, world, B,
-                            heads, N, HEAD_DIM, _cur_stream(device))
-    if rc != VA3D_OK:
-        raise VA3DError("va3d_ring_pass", rc)
+    _run("va3d_ring_pass", _device(device), ctypes.c_void_p(region), ctypes.c_void_p(next_region),
+         buf, world, B, heads, N, HEAD_DIM, _cur_stream(device))
 
 
 def ring_free(prev_region, device=None):
-    rc = lib.va3d_ring_free(ctypes.c_void_p(prev_region), _cur_stream(device))
-    if rc != VA3D_OK:
-        raise VA3DError("va3d_ring_free", rc)
+    _run("va3d_ring_free", _device(device), ctypes.c_void_p(prev_region), _cur_stream(device))
 
 
 def ring_wait(region, counter, count, world, B, heads, N, device=None):
-    rc = lib.va3d_ring_wait(ctypes.c_void_p(region), counter, int(count), world, B, heads, N,
-                            HEAD_DIM, _cur_stream(device))
-    if rc != VA3D_OK:
-        raise VA3DError("va3d_ring_wait", rc)
+    _run("va3d_ring_wait", _device(device), ctypes.c_void_p(region), counter, int(count), world, B,
+         heads, N, HEAD_DIM, _cur_stream(device))
 
 
 def ring_merge(o_blk, lse_blk, acc, lse_in, lse_out, *, first, out=None):
@@ -520,10 +542,10 @@ def ring_merge(o_blk, lse_blk, acc, lse_in, lse_out, *, first, out=None):
             raise ValueError(f"{nm} must be a contiguous float32 [B, heads, n] tensor")
     if out is not None:
         _check(out, "out", o_blk.shape)
-    rc = lib.va3d_ring_merge(_ptr(o_blk), _ptr(lse_blk), _ptr(acc), None if first else _ptr(lse_in),
-                             _ptr(lse_out), _ptr(out), B, H, n, 1 if first else 0, _stream(o_blk))
-    if rc != VA3D_OK:
-        raise VA3DError("va3d_ring_merge", rc)
+    _same_device(o_blk, lse_blk, acc, lse_out, out, None if first else lse_in)
+    _run("va3d_ring_merge", o_blk.device, _ptr(o_blk), _ptr(lse_blk), _ptr(acc),
+         None if first else _ptr(lse_in), _ptr(lse_out), _ptr(out), B, H, n, 1 if first else 0,
+         _stream(o_blk))
 
 
 class _DeviceMemory:

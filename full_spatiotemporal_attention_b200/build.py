@@ -1,4 +1,11 @@
-"""Build libva3d.so in-tree with nvcc for sm_100a (B200)."""
+"""Build libva3d.so in-tree with nvcc for sm_100a (B200).
+
+The library is rebuilt whenever the SHA-256 of its sources (the .cu file, the
+kernel headers and include/va3d.h) and of the nvcc command line differs from
+the one recorded next to it at its last build (``libva3d.so.stamp``), so a
+library built from other sources is never reused, whatever the file times.
+"""
+import hashlib
 import os
 import subprocess
 import sys
@@ -7,9 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libva3d.so")
+STAMP = LIB + ".stamp"
 SOURCES = [os.path.join(CSRC, "va3d_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
-    os.path.join(ROOT, "include", "va3d.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -20,6 +26,23 @@ NVCC_FLAGS = [
 ]
 
 
+def deps():
+    headers = sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))
+    return SOURCES + [os.path.join(CSRC, f) for f in headers] + [
+        os.path.join(ROOT, "include", "va3d.h")]
+
+
+def source_hash(flags=None):
+    """SHA-256 over the nvcc flags and every source file (name and bytes)."""
+    h = hashlib.sha256()
+    h.update(" ".join(NVCC_FLAGS if flags is None else flags).encode())
+    for d in deps():
+        h.update(os.path.relpath(d, ROOT).encode() + b"\0")
+        with open(d, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def nvcc():
     cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
     path = os.path.join(cuda, "bin", "nvcc")
@@ -27,15 +50,16 @@ def nvcc():
 
 
 def up_to_date():
-    if not os.path.exists(LIB):
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(d) <= t for d in DEPS)
+    with open(STAMP) as f:
+        return f.read().strip() == source_hash()
 
 
 def build(force=False, verbose=False):
     if not force and up_to_date():
         return LIB
+    digest = source_hash()
     cmd = [nvcc()] + NVCC_FLAGS + ["-o", LIB] + SOURCES
     res = subprocess.run(cmd, capture_output=True, text=True)
     log = os.path.join(HERE, "build.log")
@@ -44,6 +68,8 @@ def build(force=False, verbose=False):
     if res.returncode != 0:
         sys.stderr.write(res.stderr)
         raise RuntimeError(f"nvcc failed (see {log})")
+    with open(STAMP, "w") as f:
+        f.write(digest + "\n")
     if verbose:
         sys.stderr.write(res.stderr)
     return LIB

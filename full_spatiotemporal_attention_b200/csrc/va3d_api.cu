@@ -62,14 +62,64 @@ int check_sizes(int B, int heads, int N, int head_dim) {
     return VA3D_OK;
 }
 
+// Per-device facts every launch needs (architecture check, SM count, the
+// dynamic shared-memory limit already granted to each kernel), looked up
+// once per device under a mutex instead of on every call.
+constexpr int kMaxDevices = 64;
+enum KernelSlot { K_ATTN2, K_ATTN1, K_TEMP32R, K_TEMP32K, K_TEMP64R, K_TEMP64K, NUM_KERNEL_SLOTS };
+
+struct DeviceInfo {
+    int state;                     // 0 unknown, 1 sm_100, 2 other architecture
+    int sms;
+    int smem_set[NUM_KERNEL_SLOTS];   // dynamic shared memory granted so far
+};
+DeviceInfo g_devices[kMaxDevices] = {};
+std::mutex g_devices_mutex;
+
+int current_device(int *dev) {
+    if (cudaGetDevice(dev) != cudaSuccess) return VA3D_ERR_CUDA;
+    if (*dev < 0 || *dev >= kMaxDevices) return VA3D_ERR_UNSUPPORTED;
+    return VA3D_OK;
+}
+
 int check_device() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return VA3D_ERR_CUDA;
-    int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    int dev = 0, rc;
+    if ((rc = current_device(&dev)) != VA3D_OK) return rc;
+    std::lock_guard<std::mutex> lock(g_devices_mutex);
+    DeviceInfo &d = g_devices[dev];
+    if (d.state == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return VA3D_ERR_CUDA;
+        d.sms = sms;
+        d.state = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    return d.state == 1 ? VA3D_OK : VA3D_ERR_DEVICE;
+}
+
+// SM count of the current device (after check_device() succeeded on it).
+int device_sms(int *sms) {
+    int dev = 0, rc;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    if ((rc = current_device(&dev)) != VA3D_OK) return rc;
+    std::lock_guard<std::mutex> lock(g_devices_mutex);
+    *sms = g_devices[dev].sms;
+    return VA3D_OK;
+}
+
+// Grant `kernel` (slot `slot`) at least `bytes` of dynamic shared memory on
+// the current device; the attribute is set only when the need grows.
+int grant_smem(const void *kernel, int slot, int bytes) {
+    int dev = 0, rc;
+    if ((rc = current_device(&dev)) != VA3D_OK) return rc;
+    std::lock_guard<std::mutex> lock(g_devices_mutex);
+    int &set = g_devices[dev].smem_set[slot];
+    if (bytes <= set) return VA3D_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return VA3D_ERR_CUDA;
-    if (major != 10 || minor != 0) return VA3D_ERR_DEVICE;
+    set = bytes;
     return VA3D_OK;
 }
 
@@ -279,10 +329,8 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
     // One CTA per SM.  If the last wave of tiles would fill at most half of the
     // SMs and every tile has at least two 128-key steps, each of its tiles is
     // covered by two units over half of the keys instead.
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return VA3D_ERR_CUDA;
+    int sms = 0;
+    if ((rc = device_sms(&sms)) != VA3D_OK) return rc;
     const long long tiles = static_cast<long long>(BH) * n_seg * a.q_blocks;
     const long long resident = static_cast<long long>(sms) * (nq == 2 ? fa::KCfg<2>::kMinBlocks
                                                                       : fa::KCfg<1>::kMinBlocks);
@@ -298,16 +346,16 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
     if (units > 0x7fffffffll) return VA3D_ERR_UNSUPPORTED;
     if (nq == 2) {
         using C = fa::KCfg<2>;
-        if (cudaFuncSetAttribute(fa::attn_fwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes) != cudaSuccess)
-            return VA3D_ERR_CUDA;
+        if ((rc = grant_smem(reinterpret_cast<const void *>(fa::attn_fwd_kernel<2>), K_ATTN2,
+                             C::kSmemBytes)) != VA3D_OK)
+            return rc;
         fa::attn_fwd_kernel<2><<<static_cast<unsigned>(units), C::kThreads, C::kSmemBytes, st>>>(
             mq, mk, mv, a);
     } else {
         using C = fa::KCfg<1>;
-        if (cudaFuncSetAttribute(fa::attn_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes) != cudaSuccess)
-            return VA3D_ERR_CUDA;
+        if ((rc = grant_smem(reinterpret_cast<const void *>(fa::attn_fwd_kernel<1>), K_ATTN1,
+                             C::kSmemBytes)) != VA3D_OK)
+            return rc;
         fa::attn_fwd_kernel<1><<<static_cast<unsigned>(units), C::kThreads, C::kSmemBytes, st>>>(
             mq, mk, mv, a);
     }
@@ -316,10 +364,8 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
 
 template <int MAXT, bool kRawK>
 int launch_temporal_t(const tp::TemporalArgs &a, cudaStream_t st) {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return VA3D_ERR_CUDA;
+    int sms = 0, rc;
+    if ((rc = device_sms(&sms)) != VA3D_OK) return rc;
     // Warps per block and blocks per SM from the shared-memory budget; the
     // grid is persistent (at most the resident blocks), each warp strides
     // over (batch*head, position) tasks.
@@ -329,9 +375,10 @@ int launch_temporal_t(const tp::TemporalArgs &a, cudaStream_t st) {
     const int warps = std::max(1, std::min(tp::Cfg<MAXT>::kMaxWarps, budget / warp_bytes));
     const int smem = table_bytes + warps * warp_bytes;
     const int per_sm = std::max(1, std::min(4, (216 * 1024) / smem));
-    if (cudaFuncSetAttribute(tp::temporal_kernel<MAXT, kRawK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-        return VA3D_ERR_CUDA;
+    constexpr int slot = MAXT <= 32 ? (kRawK ? K_TEMP32R : K_TEMP32K) : (kRawK ? K_TEMP64R : K_TEMP64K);
+    if ((rc = grant_smem(reinterpret_cast<const void *>(tp::temporal_kernel<MAXT, kRawK>), slot, smem)) !=
+        VA3D_OK)
+        return rc;
     const long long tasks = static_cast<long long>(a.BH) * a.HW;
     const long long need = (tasks + warps - 1) / warps;
     const long long blocks = std::min<long long>(need, static_cast<long long>(sms) * per_sm);
@@ -371,16 +418,28 @@ struct Prepared {
     SplitScratch split;
 };
 
+// Workspace bytes a call cannot do without: the angle table and, unless the
+// keys come rotated, the rotated keys.  The split scratch behind them is
+// optional (split_scratch() sizes it from what is left).
+size_t required_workspace_bytes(int B, int heads, int N, const va3d_grid_t *grid, unsigned flags) {
+    return table_bytes(grid) + ((flags & VA3D_K_ROTATED) ? 0 : tensor_bytes(B, heads, N));
+}
+
+// split_optional: accept a workspace that holds only the required part (the
+// built-in scratch of the no-allocation entry point); the public entry
+// points ask for the full va3d_workspace_bytes().
 int prepare(const void *q, const void *k, const void *v, int B, int heads, int N, int head_dim,
             const va3d_grid_t *grid, float softmax_scale, unsigned flags, void *workspace,
-            size_t workspace_bytes, bool need_k_rot, cudaStream_t st, Prepared *out) {
+            size_t workspace_bytes, bool need_k_rot, cudaStream_t st, Prepared *out,
+            bool split_optional = false) {
     int rc;
     if ((rc = check_sizes(B, heads, N, head_dim)) != VA3D_OK) return rc;
     if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
     if (q == nullptr || k == nullptr || v == nullptr) return VA3D_ERR_INVALID;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return VA3D_ERR_ALIGNMENT;
     if (flags & ~static_cast<unsigned>(VA3D_K_ROTATED)) return VA3D_ERR_INVALID;
-    const size_t need = va3d_workspace_bytes(B, heads, N, head_dim, grid, flags);
+    const size_t need = split_optional ? required_workspace_bytes(B, heads, N, grid, flags)
+                                       : va3d_workspace_bytes(B, heads, N, head_dim, grid, flags);
     if (workspace == nullptr || workspace_bytes < need) return VA3D_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return VA3D_ERR_ALIGNMENT;
     if ((rc = check_device()) != VA3D_OK) return rc;
@@ -389,7 +448,7 @@ int prepare(const void *q, const void *k, const void *v, int B, int heads, int N
     out->tab = static_cast<const float2 *>(workspace);
     out->scale = softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(double(head_dim)));
     // workspace: [angle table | rotated keys (unless given) | split scratch]
-    size_t used = table_bytes(grid) + ((flags & VA3D_K_ROTATED) ? 0 : tensor_bytes(B, heads, N));
+    size_t used = required_workspace_bytes(B, heads, N, grid, flags);
     out->split = split_scratch(used < workspace_bytes ? static_cast<uint8_t *>(workspace) + used : nullptr,
                                used < workspace_bytes ? workspace_bytes - used : 0);
     if ((rc = launch_table(static_cast<float2 *>(workspace), out->split.count, out->split.capacity,
@@ -467,21 +526,37 @@ int rope3d_apply(const va3d_bf16 *x, va3d_bf16 *y, int B, int heads, int N, int 
     return launch_rope(x, y, B * heads, N, make_rope_params(grid), static_cast<cudaStream_t>(stream));
 }
 
-int attn3d_full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *o,
-                    float *lse, int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
-                    float softmax_scale, unsigned flags, void *workspace, size_t workspace_bytes,
-                    void *stream) {
-    TraceRange trace("va3d.attn3d_full_fwd");
+}  // extern "C"
+
+namespace {
+
+int full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *o, float *lse,
+             int B, int heads, int N, int head_dim, const va3d_grid_t *grid, float softmax_scale,
+             unsigned flags, void *workspace, size_t workspace_bytes, void *stream,
+             bool split_optional) {
     if (o == nullptr) return VA3D_ERR_INVALID;
     if (!aligned16(o) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return VA3D_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Prepared p;
     int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
-                     workspace_bytes, true, st, &p);
+                     workspace_bytes, true, st, &p, split_optional);
     if (rc != VA3D_OK) return rc;
     return launch_attn(q, p.k_rot, v, o, lse, B * heads, N, N, N, N, 1, true, p.rp, p.tab, p.scale,
                        p.split, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn3d_full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf16 *o,
+                    float *lse, int B, int heads, int N, int head_dim, const va3d_grid_t *grid,
+                    float softmax_scale, unsigned flags, void *workspace, size_t workspace_bytes,
+                    void *stream) {
+    TraceRange trace("va3d.attn3d_full_fwd");
+    return full_fwd(q, k, v, o, lse, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
+                    workspace_bytes, stream, false);
 }
 
 int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
@@ -853,30 +928,68 @@ int va3d_ring_merge(const va3d_bf16 *o_blk, const float *lse_blk, float *acc, co
 // device memory.  Its scratch is this one static device array; every GPU that
 // loads the library holds it until the process exits.  In host code the
 // array's name is only a host-side stand-in, so the device address is looked
-// up with cudaGetSymbolAddress, once per device with that device current, and
-// cached.  Nothing in the scratch needs to start at zero: the table and the
-// rotated keys are written before they are read on every call.
+// up with cudaGetSymbolAddress with the device current, and cached.  The
+// address belongs to the CUDA context that was current at the lookup, so the
+// cache is keyed by that context's unique id (cuCtxGetId): a call under
+// another context (a driver-API context of the caller's, or the primary
+// context recreated after cudaDeviceReset) looks the address up again.
+// Nothing in the scratch needs to start at zero: the table and the rotated
+// keys are written before they are read on every call, and the split-tail
+// counters behind them are cleared by the table kernel of every call.
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[VA3D_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
-void *g_noalloc_addr[kMaxDevices] = {};
+struct NoallocSlot {
+    unsigned long long ctx_id;   // 0: not looked up yet
+    void *addr;
+};
+NoallocSlot g_noalloc_slot[kMaxDevices] = {};
+
+// Unique id of the calling thread's current context; 0 when no context is
+// current yet (the runtime creates the primary one on its first use).
+int current_context_id(unsigned long long *id) {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    if (get_current == nullptr || get_id == nullptr) return VA3D_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return VA3D_ERR_CUDA;
+    *id = 0;
+    if (ctx != nullptr && get_id(ctx, id) != CUDA_SUCCESS) return VA3D_ERR_CUDA;
+    return VA3D_OK;
+}
 
 int noalloc_scratch(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return VA3D_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return VA3D_ERR_UNSUPPORTED;
+    int dev = 0, rc;
+    if ((rc = current_device(&dev)) != VA3D_OK) return rc;
+    unsigned long long ctx_id = 0;
+    if ((rc = current_context_id(&ctx_id)) != VA3D_OK) return rc;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_addr[dev] == nullptr) {
+    NoallocSlot &slot = g_noalloc_slot[dev];
+    if (ctx_id == 0 || slot.ctx_id != ctx_id || slot.addr == nullptr) {
+        // (the lookup itself makes the primary context current if none was)
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
             return VA3D_ERR_CUDA;
-        g_noalloc_addr[dev] = ptr;
+        if (ctx_id == 0 && (rc = current_context_id(&ctx_id)) != VA3D_OK) return rc;
+        slot.ctx_id = ctx_id;
+        slot.addr = ptr;
     }
-    *out = g_noalloc_addr[dev];
+    *out = slot.addr;
     return VA3D_OK;
 }
 
@@ -886,14 +999,18 @@ extern "C" int attn3d_full_fwd_noalloc(const va3d_bf16 *q, const va3d_bf16 *k, c
                                        va3d_bf16 *o, float *lse, int B, int heads, int N,
                                        int head_dim, const va3d_grid_t *grid, float softmax_scale,
                                        unsigned flags, void *stream) {
-    const size_t need = va3d_workspace_bytes(B, heads, N, head_dim, grid, flags);
-    if (need == 0)   // invalid sizes or grid: report them exactly as the workspace entry does
-        return attn3d_full_fwd(q, k, v, o, lse, B, heads, N, head_dim, grid, softmax_scale, flags,
-                               nullptr, 0, stream);
-    if (need > VA3D_NOALLOC_SCRATCH_BYTES) return VA3D_ERR_SCRATCH_LIMIT;
+    TraceRange trace("va3d.attn3d_full_fwd_noalloc");
+    int rc;
+    // invalid sizes or grid: report them exactly as the workspace entry does
+    if ((rc = check_sizes(B, heads, N, head_dim)) != VA3D_OK) return rc;
+    if ((rc = check_grid(grid, N, head_dim)) != VA3D_OK) return rc;
+    if (flags & ~static_cast<unsigned>(VA3D_K_ROTATED)) return VA3D_ERR_INVALID;
+    // Only the angle table and the rotated keys must fit; the split-tail
+    // scratch takes what is left of the array (none: the last wave runs whole).
+    if (required_workspace_bytes(B, heads, N, grid, flags) > VA3D_NOALLOC_SCRATCH_BYTES)
+        return VA3D_ERR_SCRATCH_LIMIT;
     void *scratch = nullptr;
-    const int rc = noalloc_scratch(&scratch);
-    if (rc != VA3D_OK) return rc;
-    return attn3d_full_fwd(q, k, v, o, lse, B, heads, N, head_dim, grid, softmax_scale, flags,
-                           scratch, VA3D_NOALLOC_SCRATCH_BYTES, stream);
+    if ((rc = noalloc_scratch(&scratch)) != VA3D_OK) return rc;
+    return full_fwd(q, k, v, o, lse, B, heads, N, head_dim, grid, softmax_scale, flags, scratch,
+                    VA3D_NOALLOC_SCRATCH_BYTES, stream, true);
 }

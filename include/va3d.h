@@ -243,21 +243,28 @@ int attn_cross_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, v
  * slow.  (The pages have no counterpart; this is a property of the library.)
  *
  * Same arguments, results and errors as attn3d_full_fwd, minus the workspace.
- * Its scratch (angle table and, unless VA3D_K_ROTATED, the rotated keys) lives
- * in one static device array of VA3D_NOALLOC_SCRATCH_BYTES (64 MiB) built into
- * the library; every GPU that loads the library holds that array until the
- * process exits.  A call whose scratch need, va3d_workspace_bytes(B, heads,
- * N, head_dim, grid, flags), exceeds 64 MiB returns VA3D_ERR_SCRATCH_LIMIT
- * and launches nothing (without VA3D_K_ROTATED that is about
- * B*heads*N <= 262,000 rows).  The function calls no allocator.
+ * Its scratch lives in one static device array of VA3D_NOALLOC_SCRATCH_BYTES
+ * (64 MiB) built into the library; every GPU that loads the library holds
+ * that array until the process exits.  The array must hold the angle table
+ * and, unless VA3D_K_ROTATED, the rotated keys (B*heads*N*256 bytes); a call
+ * whose table plus rotated keys exceed 64 MiB returns VA3D_ERR_SCRATCH_LIMIT
+ * and launches nothing.  Without VA3D_K_ROTATED that allows up to
+ * B*heads*N of about 262,000 rows (e.g. 7 heads of 32,760 tokens, not 8);
+ * with it, any size the workspace entry takes.  Whatever is left of the
+ * array after those parts serves as scratch for splitting the last partial
+ * wave of query tiles; when too little is left, that wave runs whole (same
+ * results, a little slower).  The function calls no allocator.
  *
  * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array, and each call overwrites the
- * parts it reads before reading them, so leftovers of the previous call do no
- * harm; but calls that overlap in time on the GPU (different streams, or
- * different host threads, without ordering between them) race on the array
- * and give wrong results.  Order them on one stream or synchronise.
+ * device current) and caches it per CUDA context (by the context's unique
+ * id), so a call under another context, or after cudaDeviceReset, looks it
+ * up again; make the first call of each context before any stream capture.
+ * All calls share the one array, and each call writes the parts it reads
+ * before reading them (the table, the rotated keys and the split counters),
+ * so leftovers of the previous call do no harm; but calls that overlap in
+ * time on the GPU (different streams, or different host threads, without
+ * ordering between them) race on the array and give wrong results.  Order
+ * them on one stream or synchronise.
  */
 int attn3d_full_fwd_noalloc(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v,
                             va3d_bf16 *o, float *lse, int B, int heads, int N, int head_dim,

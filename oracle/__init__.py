@@ -7,11 +7,12 @@ anything here, and this package never imports the product.
 
 Two layers:
 
-* page helpers in pure Python, restating the closed forms the handbook page
+* page helpers in pure Python, written from the closed forms the handbook page
   ("A video model's architecture: spatiotemporal attention and the 3D VAE")
-  prints: ``video_tokens`` (section "The latents: the extra time axis"),
-  ``attn_flops`` and ``linear_flops`` (section "How attention sees time:
-  factorised or full"), ``rope_3d_dims`` (section "Position: RoPE in three
+  states: ``latent_shape``, ``patch_grid``, ``token_count`` and
+  ``token_width`` (section "The latents: the extra time axis"),
+  ``attention_flops`` and ``linear_flops`` (section "How attention sees time:
+  factorised or full"), ``rope_ranges`` (section "Position: RoPE in three
   dimensions");
 * the fp64 C oracle (``va3d_oracle.c``) for RoPE and attention, reached with
   ctypes: ``rope3d``, ``attention`` (full, spatial, temporal, joint),
@@ -21,7 +22,6 @@ Two layers:
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 import subprocess
 from dataclasses import dataclass
@@ -37,58 +37,74 @@ MODES = {"full": FULL, "spatial": SPATIAL, "temporal": TEMPORAL}
 
 
 # ---------------------------------------------------------------------------
-# Page helpers (closed forms printed by the handbook page)
+# Page helpers: the handbook's closed forms for the token grid and the cost
+# model, written from its formulas
 # ---------------------------------------------------------------------------
 
-def video_tokens(frames, h, w, ft=4, fs=8, pt=1, ps=2, latent_ch=16):
-    """Latent grid, token count and token width for a clip.
-
-    Handbook, "The latents: the extra time axis": the first frame is encoded
-    on its own and every ``ft`` further frames become one latent frame;
-    space shrinks by ``fs``; patches of ``pt x ps x ps`` become tokens (floor
-    division, as the page's function does).  Returns
-    ``((T, H_lat, W_lat), tokens, token_dim)`` where ``H_lat, W_lat`` are the
-    latent (pre-patch) sizes, as the page prints them.
-    """
-    T = 1 + (frames - 1) // ft
-    H, W = h // fs, w // fs
-    tokens = (T // pt) * (H // ps) * (W // ps)
-    return (T, H, W), tokens, latent_ch * pt * ps * ps
+# Handbook, "The latents: the extra time axis": the causal 3D VAE keeps the
+# first frame and folds every 4 further frames into one latent frame, divides
+# height and width by 8, and emits 16 channels; the DiT then cuts latents into
+# 1 x 2 x 2 patches (one token each).
+VAE_TIME_STRIDE = 4
+VAE_SPACE_STRIDE = 8
+LATENT_CHANNELS = 16
+PATCH = (1, 2, 2)
 
 
-def patch_grid(frames, h, w, ft=4, fs=8, pt=1, ps=2):
-    """Post-patch token grid (T', H', W') = (T/pt, H_lat/ps, W_lat/ps)."""
-    (T, H, W), _, _ = video_tokens(frames, h, w, ft, fs, pt, ps)
-    return T // pt, H // ps, W // ps
+def latent_shape(frames, height, width):
+    """Latent (T, H_lat, W_lat) of a clip: 1 + floor((frames - 1) / 4) frames
+    and floor(height / 8) x floor(width / 8) (the page divides with floors)."""
+    return (1 + (frames - 1) // VAE_TIME_STRIDE, height // VAE_SPACE_STRIDE,
+            width // VAE_SPACE_STRIDE)
 
 
-def attn_flops(T, H, W, d, layers, mode):
-    """Attention FLOPs per denoising step (handbook, "How attention sees time").
+def patch_grid(frames, height, width):
+    """Token grid (T', H', W'): the latent shape divided by the patch size."""
+    return tuple(n // p for n, p in zip(latent_shape(frames, height, width), PATCH))
 
-    ``T, H, W`` are latent sizes (patch 2 applied inside, as on the page);
-    ``d`` is the model width (heads x head_dim).  Factorised: spatial term
-    T*4*n_sp^2*d plus temporal term n_sp*4*T^2*d; full: 4*(T*n_sp)^2*d.
-    """
-    n_sp = (H // 2) * (W // 2)
-    if mode == "factorised":
-        per_layer = T * 4 * n_sp ** 2 * d + n_sp * 4 * T ** 2 * d
-    elif mode == "full":
-        per_layer = 4 * (T * n_sp) ** 2 * d
+
+def token_count(frames, height, width):
+    """Video tokens T' * H' * W' of a clip."""
+    t, h, w = patch_grid(frames, height, width)
+    return t * h * w
+
+
+def token_width():
+    """Values per token before the patch embedding: channels x patch volume (64)."""
+    return LATENT_CHANNELS * PATCH[0] * PATCH[1] * PATCH[2]
+
+
+def attention_flops(grid, width, layers, mode):
+    """Attention FLOPs of one denoising step (handbook, "How attention sees
+    time: factorised or full").  ``grid`` is the token grid (T', H', W'),
+    ``width`` the model width (heads x head_dim).  Full attention costs
+    4 (T'H'W')^2 width per layer; the factorised form costs 4 width
+    (T' (H'W')^2 + H'W' T'^2): T' spatial sequences of H'W' tokens plus H'W'
+    temporal sequences of T' tokens."""
+    t, h, w = grid
+    s = h * w
+    if mode == "full":
+        per_layer = 4 * (t * s) ** 2 * width
+    elif mode == "factorised":
+        per_layer = 4 * width * (t * s * s + s * t * t)
     else:
-        raise ValueError(mode)
+        raise ValueError(f"mode must be 'full' or 'factorised', not {mode!r}")
     return layers * per_layer
 
 
-def linear_flops(tokens, d, layers):
-    """Linear-layer FLOPs per step, 24*N*d^2 per layer (same section)."""
-    return layers * 24 * tokens * d * d
+def linear_flops(tokens, width, layers):
+    """Linear-layer FLOPs of one step, 24 tokens width^2 per layer (same section)."""
+    return layers * 24 * tokens * width * width
 
 
-def rope_3d_dims(head_dim=128, axes=(16, 56, 56)):
-    """Head-dim allocation of 3D RoPE; the three ranges must fill the head
-    (handbook, "Position: RoPE in three dimensions")."""
-    assert sum(axes) == head_dim
-    return {"t": axes[0], "h": axes[1], "w": axes[2]}
+def rope_ranges(split, head_dim=128):
+    """Head-dim ranges [start, end) turned by t, h and w (handbook, "Position:
+    RoPE in three dimensions"): three contiguous ranges in t, h, w order that
+    together fill the head, each of an even width (it holds whole pairs)."""
+    if len(split) != 3 or sum(split) != head_dim or any(d < 0 or d % 2 for d in split):
+        raise ValueError(f"a 3D RoPE split needs three even widths summing to {head_dim}: {split}")
+    d_t, d_h, _ = split
+    return {"t": (0, d_t), "h": (d_t, d_t + d_h), "w": (d_t + d_h, head_dim)}
 
 
 def token_coords(i, T, H, W):
@@ -285,18 +301,3 @@ def cross_attention(q_bits, k_bits, v_bits, rows=None, scale=None, want_lse=Fals
     if rc != 0:
         raise ValueError(f"oracle_cross_attention rejected the arguments ({rc})")
     return (out, lse) if want_lse else out
-
-
-def full_flops(N, heads, head_dim=128):
-    """4*N^2*d*heads: the FLOP count of one full-attention forward."""
-    return 4 * N * N * head_dim * heads
-
-
-def factorised_flops(T, H, W, heads, head_dim=128):
-    """4*d*heads*(T*(HW)^2 + HW*T^2): spatial plus temporal pass."""
-    hw = H * W
-    return 4 * head_dim * heads * (T * hw * hw + hw * T * T)
-
-
-def default_scale(head_dim=128):
-    return 1.0 / math.sqrt(head_dim)

@@ -27,7 +27,7 @@
  *    cross-attention (queries from the video tokens, keys and values from
  *    the text encoder's tokens, which the step does not update).
  *
- * Readings where the pages are silent (each is listed in the design notes):
+ * Readings where the pages are silent:
  *  - pairs are adjacent (2j, 2j+1) inside each axis range;
  *  - each axis has its own frequency ladder theta^(-2j/d_a), theta = 10000;
  *  - ranges are ordered t, h, w at offsets 0, d_t, d_t + d_h;

@@ -94,10 +94,10 @@ def test_token_table_matches_printed(golden_dir):
     for line in _rows(os.path.join(golden_dir, "token_table.txt")):
         clip, lat, tokens, dim, ratio = [p.split() for p in line.split("|")]
         frames, h, w = map(int, clip)
-        (T, H, W), n, d = oracle.video_tokens(frames, h, w)
-        assert (T, H, W) == tuple(map(int, lat))
+        assert oracle.latent_shape(frames, h, w) == tuple(map(int, lat))
+        n = oracle.token_count(frames, h, w)
         assert n == int(tokens[0])
-        assert d == int(dim[0])
+        assert oracle.token_width() == int(dim[0])
         assert round(n / 4096) == int(ratio[0])
 
 
@@ -106,9 +106,9 @@ def test_flops_table_matches_printed(golden_dir):
         left, right = line.split("|")
         frames, h, w, d, layers = map(int, left.split())
         fact, full, ratio, lin = map(int, right.split())
-        (T, H, W), n, _ = oracle.video_tokens(frames, h, w)
-        f1 = oracle.attn_flops(T, H, W, d, layers, "factorised")
-        f2 = oracle.attn_flops(T, H, W, d, layers, "full")
+        grid, n = oracle.patch_grid(frames, h, w), oracle.token_count(frames, h, w)
+        f1 = oracle.attention_flops(grid, d, layers, "factorised")
+        f2 = oracle.attention_flops(grid, d, layers, "full")
         assert round(f1 / 1e12) == fact
         assert round(f2 / 1e12) == full
         assert round(f2 / f1) == ratio
@@ -123,18 +123,18 @@ def test_page_arithmetic(golden_dir):
     pixels = 81 * 832 * 480
     assert pixels == vals["pixels"][0]
     assert round(pixels ** 2 / 1e15, 3) == vals["raw_pairs_quadrillion"][0]
-    _, n, _ = oracle.video_tokens(81, 480, 832)
+    n = oracle.token_count(81, 480, 832)
     assert n == vals["tokens"][0]
     assert int(pixels ** 2 / n ** 2) == vals["attention_cut"][0]
     assert round(pixels ** 2 * 2 / 1e12) == vals["raw_score_TB_one_head"][0]
     assert round(n * n * 2 / 1e9, 2) == vals["score_GB_one_head"][0]
     assert round(pixels * 3 / 1e6, 2) == vals["raw_floats_M"][0]
-    (T, H, W), _, _ = oracle.video_tokens(81, 480, 832)
-    assert round(T * H * W * 16 / 1e6, 2) == vals["latent_floats_M"][0]
+    T, H, W = oracle.latent_shape(81, 480, 832)
+    assert round(T * H * W * oracle.LATENT_CHANNELS / 1e6, 2) == vals["latent_floats_M"][0]
     assert [d // 2 for d in (44, 42, 42)] == vals["rope_pairs_t_h_w"]
     # exercises: 480p -> 720p growth and reference-image tokens
-    _, n480, _ = oracle.video_tokens(81, 480, 832)
-    _, n720, _ = oracle.video_tokens(81, 720, 1280)
+    n480 = oracle.token_count(81, 480, 832)
+    n720 = oracle.token_count(81, 720, 1280)
     assert (n480, n720) == (vals["tokens_480p"][0], vals["tokens_720p"][0])
     assert round(n720 / n480, 1) == vals["token_growth"][0]
     assert round((n720 / n480) ** 2, 1) == vals["attention_growth"][0]
@@ -153,10 +153,9 @@ def test_page_arithmetic(golden_dir):
 
 def test_frame_rule_examples():
     # handbook VAE example: 9 frames of 32x32 -> 3 latent frames of 4x4 (compression 8)
-    (T, H, W), _, _ = oracle.video_tokens(9, 32, 32)
-    assert (T, H, W) == (3, 4, 4)
+    assert oracle.latent_shape(9, 32, 32) == (3, 4, 4)
     # CogVideoX guide: 49 frames -> 13 latent frames
-    assert oracle.video_tokens(49, 480, 720)[0][0] == 13
+    assert oracle.latent_shape(49, 480, 720)[0] == 13
     # the configurations of this build
     assert oracle.patch_grid(81, 480, 832) == (21, 30, 52)
     assert oracle.patch_grid(81, 720, 1280) == (21, 45, 80)
@@ -164,11 +163,14 @@ def test_frame_rule_examples():
     assert oracle.patch_grid(17, 480, 832) == (5, 30, 52)
 
 
-def test_rope_dims_allocator():
-    assert oracle.rope_3d_dims() == {"t": 16, "h": 56, "w": 56}
-    assert oracle.rope_3d_dims(128, (44, 42, 42))["t"] == 44
-    with pytest.raises(AssertionError):
-        oracle.rope_3d_dims(128, (44, 42, 40))
+def test_rope_ranges():
+    # HunyuanVideo's (16, 56, 56) and Wan2.1's (44, 42, 42) both fill the head
+    assert oracle.rope_ranges((16, 56, 56)) == {"t": (0, 16), "h": (16, 72), "w": (72, 128)}
+    r = oracle.rope_ranges((44, 42, 42))
+    assert [(b - a) // 2 for a, b in r.values()] == [22, 21, 21]
+    for bad in ((44, 42, 40), (43, 43, 42), (128,), (64, 64, 0, 0)):
+        with pytest.raises(ValueError):
+            oracle.rope_ranges(bad)
 
 
 def test_shard_listing_matches_printed(golden_dir):

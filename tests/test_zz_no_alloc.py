@@ -87,6 +87,42 @@ def test_noalloc_after_a_different_problem_and_with_rotated_keys(va):
         assert _close(o, ref)
 
 
+def test_noalloc_limit_counts_only_the_table_and_rotated_keys(va):
+    # 7 heads x 32,760 tokens: the table and rotated keys take 58.7 MB, under
+    # the 64 MiB array; the split-tail scratch a workspace would add (34 MB
+    # for 896 tiles) is optional, so the call is taken and matches the
+    # workspace entry point.  8 heads need 67.1 MB and are refused.
+    w = si.WORKLOADS["c81f480"]
+    g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    q, k, v = (_dev(x[:, :7]) for x in si.qkv(w))
+    assert va.workspace_bytes(1, 7, w.N, g) > (64 << 20)
+    ref = va.attn3d_full_fwd(q, k, v, g)
+    for _ in range(2):
+        o = torch.full_like(q, float("nan"))
+        assert _call_noalloc(va, q, k, v, o, None, g) == 0
+        torch.cuda.synchronize()
+        assert _close(o, ref)
+    x = torch.zeros(1, 1, 1, 128, dtype=torch.bfloat16, device="cuda")
+    p = ctypes.c_void_p(x.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert va.lib.attn3d_full_fwd_noalloc(p, p, p, p, None, 1, 8, w.N, 128, ctypes.byref(g), 0.0,
+                                          0, stream) == -7
+    assert va.device_error() == 0
+
+
+def test_noalloc_binding_checks_lse(va):
+    w = si.WORKLOADS["tiny"]
+    q, k, v = (_dev(x) for x in si.qkv(w))
+    g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
+    B, H, N, _ = q.shape
+    for bad in (torch.empty((B, H, N), dtype=torch.bfloat16, device="cuda"),
+                torch.empty((B, H, N - 1), dtype=torch.float32, device="cuda"),
+                torch.empty((B, H, 2 * N), dtype=torch.float32, device="cuda")[..., ::2],
+                torch.empty((B, H, N), dtype=torch.float32)):
+        with pytest.raises(ValueError):
+            va.attn3d_full_fwd_noalloc(q, k, v, g, lse=bad)
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch(va):
     w = si.WORKLOADS["c81f480"]          # needs 100 MB of rotated keys > 64 MiB
     g = va.Grid.make(w.T, w.H, w.W, w.n_text, w.dims, w.theta)
