@@ -34,7 +34,11 @@
 // MMA issuer ping-pongs the two query tiles so that one tile's softmax
 // overlaps the other tile's QK^T and PV products; with NQ = 1 the two CTAs of
 // an SM interleave on its tensor core in the same way, and one CTA's
-// prologue and epilogue overlap the other's main loop.  Q, K, V tiles are
+// prologue and epilogue overlap the other's main loop.  A softmax group
+// publishes the P of the first 64 keys of a tile before it computes the rest,
+// so that the PV product of those keys runs while it does: a group's next
+// scores wait for its own softmax, its PV product and its QK^T product in
+// turn, and this takes the first half of the PV product off that chain.  Q, K, V tiles are
 // 128 rows x 128 bf16, loaded by TMA as two 64-column boxes with the 128-byte
 // swizzle.
 #pragma once
@@ -62,6 +66,7 @@ enum Bar {
     B_VEMPTY0, B_VEMPTY1,
     B_SFULL0, B_SFULL1,
     B_PFULL0, B_PFULL1,
+    B_PHALF0, B_PHALF1,       // the first 64 keys' P of tile g is in TMEM
     B_OFULL,
     B_DRAIN,
     B_EPI,        // split units: every softmax thread stored its partial
@@ -162,8 +167,11 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr) {
 }
 
 // Turn row `r` of a swizzled 128x128 Q tile in shared memory by 3D RoPE.
-// All 64 (cos, sin) pairs of the row are fetched first (read-only loads, all
-// in flight together), then the row is rotated in place.
+// All 64 (cos, sin) pairs of the row are formed first, from the hardware sine
+// and cosine of pos * inv_freq (absolute error ~1e-5 at the largest angles of
+// the pages' grids, far below the bf16 rounding of the turned values; 3.4k
+// cycles per tile against 9k for 64 angle-table loads per row), then the row
+// is rotated in place.
 __device__ __forceinline__ void rope_q_row(uint8_t *tile, int r, int n, const AttnArgs &a) {
     const RopeParams &rp = a.rp;
     if (n >= rp.n_video) return;   // text token or a padding row past N
@@ -173,7 +181,10 @@ __device__ __forceinline__ void rope_q_row(uint8_t *tile, int r, int n, const At
     const int w = rem - h * rp.W;
     float2 cs[64];
 #pragma unroll
-    for (int p = 0; p < 64; ++p) cs[p] = __ldg(&a.rope_tab[table_index(rp, p, t, h, w)]);
+    for (int p = 0; p < 64; ++p) {
+        const float ang = static_cast<float>(pair_pos(rp, p, t, h, w)) * rp.inv_freq[p];
+        __sincosf(ang, &cs[p].y, &cs[p].x);
+    }
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -248,6 +259,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(bar(B_SFULL1), 1);
         mbar_init(bar(B_PFULL0), BM);
         mbar_init(bar(B_PFULL1), BM);
+        mbar_init(bar(B_PHALF0), BM);
+        mbar_init(bar(B_PHALF1), BM);
         mbar_init(bar(B_OFULL), 1);
         mbar_init(bar(B_DRAIN), 1);
         mbar_init(bar(B_EPI), NQ * BM);
@@ -411,9 +424,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                            desc_kmajor(sbase + OFF_K + s * kTileBytes + off), kIdescQK, kk > 0);
                 }
             };
-            auto issue_pv = [&](int i, int s, bool acc) {
+            auto issue_pv = [&](int i, int s, bool acc, int k_lo, int k_hi) {
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
+                for (int kk = k_lo; kk < k_hi; ++kk) {
                     mma_ts(tmem + COL_O0 + i * (COL_O1 - COL_O0), tmem + COL_S0 + i * (COL_S1 - COL_S0) + kk * 8,
                            desc_mnmajor(sbase + OFF_V + s * kTileBytes + kk * 2048), kIdescPV,
                            (acc || kk > 0) ? 1u : 0u);
@@ -440,10 +453,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const int s2 = stg(j + 1);
                 const uint32_t ph2 = phs(j + 1);
                 ok = mbar_wait(bar(B_VFULL0 + s), ph, abort_flag, VA3D_DEVERR_TIMEOUT_MMA) &&
-                     mbar_wait(bar(B_PFULL0), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
+                     mbar_wait(bar(B_PHALF0), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
                 if (!ok) break;
                 tc_fence_after();
-                issue_pv(0, s, j > 0);
+                issue_pv(0, s, j > 0, 0, 4);
+                ok = mbar_wait(bar(B_PFULL0), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(0, s, true, 4, 8);
                 // one query tile: V's stage is free after this product.  (Its
                 // release must not wait for the next QK^T: with one stage the
                 // gathering loader publishes that K tile only after refilling V.)
@@ -456,10 +473,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     mma_commit(bar(B_SFULL0));
                 }
                 if constexpr (NQ == 2) {
+                    ok = mbar_wait(bar(B_PHALF1), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(1, s, j > 0, 0, 4);
                     ok = mbar_wait(bar(B_PFULL1), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(1, s, j > 0);
+                    issue_pv(1, s, true, 4, 8);
                     mma_commit(bar(B_VEMPTY0 + s));
                 }
                 if (more) {
@@ -545,23 +566,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 for (int c = 0; c < BN; ++c)
                     if (c >= kv_last_valid) s[c] = -INFINITY;
             }
-            // row maximum: four independent chains of three-input max
-            float m4[4];
+            // row maximum: a tree of three-input max (depth 5)
+            float t1[43];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float *v = s + 32 * q;
-                float m = fmax3(v[0], v[1], v[2]);
+            for (int q = 0; q < 42; ++q) t1[q] = fmax3(s[3 * q], s[3 * q + 1], s[3 * q + 2]);
+            t1[42] = fmaxf(s[126], s[127]);
+            float t2[15];
 #pragma unroll
-                for (int c = 3; c < 31; c += 2) m = fmax3(m, v[c], v[c + 1]);
-                m4[q] = fmaxf(m, v[31]);
-            }
-            const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+            for (int q = 0; q < 14; ++q) t2[q] = fmax3(t1[3 * q], t1[3 * q + 1], t1[3 * q + 2]);
+            t2[14] = t1[42];
+            float t3[5];
+#pragma unroll
+            for (int q = 0; q < 5; ++q) t3[q] = fmax3(t2[3 * q], t2[3 * q + 1], t2[3 * q + 2]);
+            const float mx = fmaxf(fmax3(t3[0], t3[1], t3[2]), fmaxf(t3[3], t3[4]));
             const float m_new = fmaxf(m_ref, mx * a.scale_log2);
             float alpha = 1.0f;
             const bool bump = m_new - m_ref > kRescaleThreshold;
             if (bump) {
                 alpha = ex2(m_ref - m_new);
                 m_ref = m_new;
+            }
+            // O must be rescaled before the first PV product of this tile
+            if (j > 0 && __any_sync(0xffffffffu, bump)) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(taO + 32 * c, ov);
+                    tmem_wait_ld();
+                    reg_fence32(ov);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                    tmem_st32(taO + 32 * c, ov);
+                }
             }
             // P = 2^(s*scale - m) in pairs; a quarter of the pairs use the FMA-pipe
             // exp2 to offload the MUFU unit (not on the masked tile, whose -inf
@@ -587,6 +624,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         pk[c] = pack_bf16x2(p.x, p.y);
                     }
                     tmem_st32(taS + 32 * hf, pk);
+                    if (hf == 0) {
+                        // the first 64 keys' P: the MMA issuer may start on them
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(bar(g ? B_PHALF1 : B_PHALF0));
+                    }
                 }
             };
             if (masked_tile)
@@ -597,19 +640,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const float2 acc23 = add2(acc[2], acc[3]);
             const float2 acc_all = add2(acc01, acc23);
             const float rowsum = acc_all.x + acc_all.y;
-            if (j > 0 && __any_sync(0xffffffffu, bump)) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t ov[32];
-                    tmem_ld32(taO + 32 * c, ov);
-                    tmem_wait_ld();
-                    reg_fence32(ov);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                    tmem_st32(taO + 32 * c, ov);
-                }
-            }
             l = l * alpha + rowsum;
             tmem_wait_st();
             tc_fence_before();
