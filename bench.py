@@ -79,12 +79,23 @@ def sustained_peak():
         return None
 
 
+def strip_comments(src):
+    """C/C++ source without its comments and with runs of white space folded,
+    so that a comment edit does not change a kernel's hash."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def kernel_source_hash(files):
+    """SHA-256 (16 hex digits) over the listed kernel sources, comments and
+    white space excluded."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "full_spatiotemporal_attention_b200", "csrc")
     for f in files:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

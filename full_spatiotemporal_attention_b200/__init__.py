@@ -39,7 +39,7 @@ SYMBOLS = ("va3d_status_string", "va3d_version", "va3d_grid_from_video",
            "va3d_region_alloc", "va3d_region_free", "va3d_ipc_export", "va3d_ipc_open",
            "va3d_ipc_close", "va3d_ulysses_scatter", "va3d_ulysses_gather", "va3d_ulysses_wait",
            "va3d_ring_region_bytes", "va3d_ring_offsets", "va3d_ring_load", "va3d_ring_pass",
-           "va3d_ring_free", "va3d_ring_wait", "va3d_ring_merge")
+           "va3d_ring_free", "va3d_ring_wait", "va3d_ring_merge", "va3d_ring_attend")
 
 
 class VA3DError(RuntimeError):
@@ -120,6 +120,7 @@ def _load():
     lib.va3d_ring_free.argtypes = [vp, vp]
     lib.va3d_ring_wait.argtypes = [vp, i, ctypes.c_ulonglong, i, i, i, i, i, vp]
     lib.va3d_ring_merge.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
+    lib.va3d_ring_attend.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     return lib
 
 
@@ -546,6 +547,32 @@ def ring_merge(o_blk, lse_blk, acc, lse_in, lse_out, *, first, out=None):
     _run("va3d_ring_merge", o_blk.device, _ptr(o_blk), _ptr(lse_blk), _ptr(acc),
          None if first else _ptr(lse_in), _ptr(lse_out), _ptr(out), B, H, n, 1 if first else 0,
          _stream(o_blk))
+
+
+def ring_attend(q_rot, k, v, acc, lse_in, lse_out, *, first, out=None, scale=None):
+    """One ring block step: attention of q_rot [B, heads, n, 128] over the
+    block k, v [B, heads, n_keys, 128] (no RoPE), merged into the fp32
+    accumulator (acc, lse_in) -> (acc, lse_out) inside the attention kernel;
+    with `out`, the merged output is also written as bf16."""
+    torch = _torch()
+    _check(q_rot, "q_rot")
+    _check(k, "k")
+    B, H, n, D = q_rot.shape
+    if k.shape[:2] != q_rot.shape[:2]:
+        raise ValueError(f"k has shape {tuple(k.shape)}, expected [{B}, {H}, n_keys, {D}]")
+    _check(v, "v", k.shape)
+    if (not isinstance(acc, torch.Tensor) or acc.dtype != torch.float32
+            or tuple(acc.shape) != (B, H, n, D) or not acc.is_contiguous()):
+        raise ValueError("acc must be a contiguous float32 tensor shaped like q_rot")
+    _check_lse(lse_out, (B, H, n))
+    if not first:
+        _check_lse(lse_in, (B, H, n))
+    if out is not None:
+        _check(out, "out", q_rot.shape)
+    _same_device(q_rot, k, v, acc, lse_out, out, None if first else lse_in)
+    _run("va3d_ring_attend", q_rot.device, _ptr(q_rot), _ptr(k), _ptr(v), _ptr(acc),
+         None if first else _ptr(lse_in), _ptr(lse_out), _ptr(out), B, H, n, k.shape[2], D,
+         float(scale or 0.0), 1 if first else 0, _stream(q_rot))
 
 
 class _DeviceMemory:

@@ -139,6 +139,15 @@ struct AttnArgs {
     int win_t, win_h, win_w;   // window size
     int nwin_h, nwin_w;        // windows along h and w
     const __nv_bfloat16 *gq, *gk, *gv;
+    // Ring merge (merge != 0, whole units only): this call is one key block
+    // of a ring; its normalised output and LSE are merged by log-sum-exp
+    // weights into the fp32 accumulator acc [rows, 128] and lse_out (natural
+    // log); merge == 1 starts them (first block), merge == 2 folds in lse_in.
+    // o, if set, receives the merged output as bf16.
+    int merge;
+    float *acc;
+    const float *lse_in;
+    float *lse_out;
 };
 
 // Natural token index of row `local` of window `seg`.
@@ -653,7 +662,59 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const float inv_l = 1.0f / l;
             const bool valid = n < seg_end;
             uint4 *dst = reinterpret_cast<uint4 *>(a.o + (static_cast<size_t>(bh) * a.N + n_out) * HD);
-            if (!split) {
+            if (a.merge) {
+                // ring block: merge into the accumulator by log-sum-exp weights
+                //   l = m + log(e^(l_in - m) + e^(l_blk - m)),
+                //   o = (e^(l_in - m) o_in + e^(l_blk - m) o_blk) / (...),
+                // in log2 units (m_ref and l give the block's log2-sum-exp)
+                const size_t row = static_cast<size_t>(bh) * a.N + n_out;
+                const float lb2 = m_ref + log2f(l);
+                float wa = 0.0f, wb = 1.0f, lo2 = lb2;
+                if (a.merge == 2 && valid) {
+                    const float la2 = a.lse_in[row] * 1.4426950408889634f;
+                    const float mm = fmaxf(la2, lb2);
+                    const float ea = ex2(la2 - mm), eb = ex2(lb2 - mm);
+                    const float inv = 1.0f / (ea + eb);
+                    wa = ea * inv;
+                    wb = eb * inv;
+                    lo2 = mm + log2f(ea + eb);
+                }
+                float4 *accp = reinterpret_cast<float4 *>(a.acc + row * HD);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(taO + 32 * c, ov);
+                    tmem_wait_ld();
+                    reg_fence32(ov);
+                    if (valid) {
+                        float x[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(ov[e]) * inv_l * wb;
+                        if (a.merge == 2) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const float4 y = accp[c * 8 + e];
+                                x[4 * e] += wa * y.x;
+                                x[4 * e + 1] += wa * y.y;
+                                x[4 * e + 2] += wa * y.z;
+                                x[4 * e + 3] += wa * y.w;
+                            }
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            accp[c * 8 + e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                        if (a.o != nullptr) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                dst[c * 4 + e] = make_uint4(pack_bf16x2(x[8 * e], x[8 * e + 1]),
+                                                            pack_bf16x2(x[8 * e + 2], x[8 * e + 3]),
+                                                            pack_bf16x2(x[8 * e + 4], x[8 * e + 5]),
+                                                            pack_bf16x2(x[8 * e + 6], x[8 * e + 7]));
+                        }
+                    }
+                }
+                if (valid) a.lse_out[row] = lo2 * 0.69314718055994531f;
+            } else if (!split) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t ov[32];

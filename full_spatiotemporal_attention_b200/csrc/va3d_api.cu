@@ -289,10 +289,19 @@ SplitScratch split_scratch(void *base, size_t bytes) {
 // attends to segment s of the keys.
 // win (optional): local 3D window size; segments are then the windows, their
 // rows gathered token by token (seg_len == kv_len == window volume).
+// merge (optional): the ring form's log-sum-exp merge into an accumulator,
+// done in the kernel's epilogue (no tile is split then).
+struct RingMerge {
+    int merge;            // 1: first block, 2: merge with lse_in
+    float *acc;
+    const float *lse_in;
+    float *lse_out;
+};
+
 int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float *lse, int BH, int N,
                 int Nkv, int seg_len, int kv_len, int n_seg, bool rope_q, const RopeParams &rp,
                 const float2 *tab, float scale, const SplitScratch &sc, cudaStream_t st,
-                const int *win = nullptr) {
+                const int *win = nullptr, const RingMerge *merge = nullptr) {
     CUtensorMap mq, mk, mv;
     int rc;
     if ((rc = make_map(&mq, q, N, BH, fa::BM)) != VA3D_OK) return rc;
@@ -326,6 +335,12 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
         a.gv = static_cast<const __nv_bfloat16 *>(v);
     }
     a.n_seg = n_seg;
+    if (merge != nullptr) {
+        a.merge = merge->merge;
+        a.acc = merge->acc;
+        a.lse_in = merge->lse_in;
+        a.lse_out = merge->lse_out;
+    }
     // One CTA per SM.  If the last wave of tiles would fill at most half of the
     // SMs and every tile has at least two 128-key steps, each of its tiles is
     // covered by two units over half of the keys instead.
@@ -337,7 +352,8 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
     const long long tail = resident > 0 ? tiles % resident : 0;
     const int n_kv = (kv_len + fa::BN - 1) / fa::BN;
     long long split = 0;
-    if (tail > 0 && 2 * tail <= resident && tail <= sc.capacity && n_kv >= 2) split = tail;
+    if (merge == nullptr && tail > 0 && 2 * tail <= resident && tail <= sc.capacity && n_kv >= 2)
+        split = tail;
     a.n_whole = static_cast<int>(tiles - split);
     a.part_o = sc.part_o;
     a.part_ml = sc.part_ml;
@@ -920,6 +936,33 @@ int va3d_ring_merge(const va3d_bf16 *o_blk, const float *lse_blk, float *acc, co
         reinterpret_cast<float4 *>(acc), lse_in, lse_out,
         out ? static_cast<uint4 *>(static_cast<void *>(out)) : nullptr, rows, first ? 1 : 0);
     return launch_status();
+}
+
+int va3d_ring_attend(const va3d_bf16 *q_rot, const va3d_bf16 *k, const va3d_bf16 *v, float *acc,
+                     const float *lse_in, float *lse_out, va3d_bf16 *out, int B, int heads,
+                     int n_rows, int n_keys, int head_dim, float softmax_scale, int first,
+                     void *stream) {
+    TraceRange trace("va3d.va3d_ring_attend");
+    int rc;
+    if ((rc = check_sizes(B, heads, n_rows, head_dim)) != VA3D_OK) return rc;
+    if ((rc = check_sizes(B, heads, n_keys, head_dim)) != VA3D_OK) return rc;
+    if (q_rot == nullptr || k == nullptr || v == nullptr || acc == nullptr || lse_out == nullptr ||
+        (!first && lse_in == nullptr) || (!first && lse_in == lse_out))
+        return VA3D_ERR_INVALID;
+    if (!aligned16(q_rot) || !aligned16(k) || !aligned16(v) || !aligned16(acc) ||
+        (out != nullptr && !aligned16(out)) || (reinterpret_cast<uintptr_t>(lse_out) & 3u) ||
+        (lse_in != nullptr && (reinterpret_cast<uintptr_t>(lse_in) & 3u)))
+        return VA3D_ERR_ALIGNMENT;
+    if ((rc = check_device()) != VA3D_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const float scale =
+        softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(double(head_dim)));
+    SplitScratch none_split = split_scratch(nullptr, 0);
+    RopeParams none;
+    std::memset(&none, 0, sizeof none);
+    const RingMerge m = {first ? 1 : 2, acc, first ? nullptr : lse_in, lse_out};
+    return launch_attn(q_rot, k, v, out, nullptr, B * heads, n_rows, n_keys, n_rows, n_keys, 1, false,
+                       none, nullptr, scale, none_split, st, nullptr, &m);
 }
 }  // extern "C"
 

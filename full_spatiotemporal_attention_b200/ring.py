@@ -7,11 +7,11 @@ One call:
 1. ``ring_load``: this rank's Q and K turned at their global positions (Q
    into ``q_rot``, K with V into the region's block buffer 0);
 2. for s = 0 .. P-1: the product of ``q_rot`` with the block in buffer
-   s % 2 (``attn_cross_fwd``, no RoPE, with its LSE), merged into an fp32
-   accumulator by log-sum-exp weights (``ring_merge``; the last merge
-   writes the bf16 output), while the same block is copied into the next
-   rank's buffer (s + 1) % 2 (``ring_pass``, on a side stream so that the
-   copy overlaps the product);
+   s % 2, merged into an fp32 accumulator by log-sum-exp weights in the
+   attention kernel's own epilogue (``ring_attend``; the last step writes the
+   bf16 output), while the same block is copied into the next rank's buffer
+   (s + 1) % 2 (``ring_pass``, on a side stream so that the copy overlaps the
+   product);
 3. ordering by the region counters: before a pass, wait until the next rank
    has finished the products that read that buffer (``free``); after a
    product, signal the previous rank (``ring_free``); before the next
@@ -80,14 +80,9 @@ class RingAttention:
                          view(self.region, v1, shape, self.device)]
             bf, f32 = torch.bfloat16, torch.float32
             self.q_rot = torch.empty(shape, dtype=bf, device=self.device)
-            self.o_blk = torch.empty(shape, dtype=bf, device=self.device)
             self.out = torch.empty(shape, dtype=bf, device=self.device)
             self.acc = torch.empty(shape, dtype=f32, device=self.device)
-            self.lse_blk = torch.empty(shape[:3], dtype=f32, device=self.device)
             self.lse = [torch.empty(shape[:3], dtype=f32, device=self.device) for _ in range(2)]
-            self.workspace = torch.empty(
-                max(va.cross_workspace_bytes(batch, heads, self.n_loc, self.n_loc), 256),
-                dtype=torch.uint8, device=self.device)
             self.side = torch.cuda.Stream(self.device) if (overlap and world > 1 and
                                                            self.device.type == "cuda") else None
         except BaseException:
@@ -123,14 +118,13 @@ class RingAttention:
                                  device=self.device)
                     va.ring_pass(self.region, self.next_region, cur, *self._shape_args(),
                                  device=self.device)
-            va.attn_cross_fwd(self.q_rot, self.kbuf[cur], self.vbuf[cur], out=self.o_blk,
-                              lse=self.lse_blk, workspace=self.workspace)
+            va.ring_attend(self.q_rot, self.kbuf[cur], self.vbuf[cur], self.acc,
+                           self.lse[(s + 1) % 2], self.lse[s % 2], first=(s == 0),
+                           out=self.out if s == P - 1 else None)
             if self.side is not None and s < P - 1:
                 torch.cuda.current_stream(self.device).wait_stream(self.side)
             if P > 1:
                 va.ring_free(self.prev_region, device=self.device)
-            va.ring_merge(self.o_blk, self.lse_blk, self.acc, self.lse[(s + 1) % 2], self.lse[s % 2],
-                          first=(s == 0), out=self.out if s == P - 1 else None)
             if s < P - 1:
                 va.ring_wait(self.region, va.RING_FULL, (c - 1) * (P - 1) + s + 1,
                              *self._shape_args(), device=self.device)

@@ -393,11 +393,12 @@ int va3d_ulysses_wait(const void *region, int phase, unsigned long long epoch, i
  * positions (positions are absolute: handbook "A video model's
  * architecture", section "Position: RoPE in three dimensions") into q_rot
  * and the region's block buffer 0, with v.  Then for steps s = 0..world-1
- * the rank attends q_rot to the block in buffer s % 2 with attn_cross_fwd
- * (no RoPE; its LSE kept), merges that partial output into an fp32
- * accumulator with va3d_ring_merge (log-sum-exp weights), and, except at the
- * last step, copies the block to the next rank's buffer (s + 1) % 2 with
- * va3d_ring_pass.  Ordering, all stream-ordered and bounded (2 s, then
+ * the rank attends q_rot to the block in buffer s % 2 and merges that
+ * partial output into an fp32 accumulator by log-sum-exp weights, in one
+ * call, va3d_ring_attend (the merge runs in the attention kernel's epilogue;
+ * the two-call form, attn_cross_fwd with its LSE then va3d_ring_merge,
+ * computes the same), and, except at the last step, copies the block to the
+ * next rank's buffer (s + 1) % 2 with va3d_ring_pass.  Ordering, all stream-ordered and bounded (2 s, then
  * VA3D_DEVERR_TIMEOUT_PEER): before va3d_ring_pass of step s of call c,
  * va3d_ring_wait(free, (c-1)*world + s) (the next rank has finished the
  * products that read that buffer); after each product va3d_ring_free on the
@@ -462,6 +463,39 @@ int va3d_ring_wait(const void *region, int counter, unsigned long long count, in
 int va3d_ring_merge(const va3d_bf16 *o_blk, const float *lse_blk, float *acc, const float *lse_in,
                     float *lse_out, va3d_bf16 *out, int B, int heads, int n_rows, int first,
                     void *stream);
+
+/*
+ * One block step of the ring form with the merge done in the attention
+ * kernel's epilogue (the product of va3d_ring_merge's inputs, without the
+ * block output ever reaching memory as bf16): the block attention
+ *   o_blk = softmax(scale * q_rot k^T) v,  l_blk = its log-sum-exp,
+ * over the n_keys keys of k, v (no RoPE: q_rot and k come turned at their
+ * global positions), merged into the accumulator as in va3d_ring_merge:
+ *   first != 0:  acc = o_blk, lse_out = l_blk;
+ *   otherwise:   with m = max(lse_in, l_blk),
+ *                acc = (e^(lse_in-m) acc + e^(l_blk-m) o_blk) / (e^(lse_in-m) + e^(l_blk-m)),
+ *                lse_out = m + log(e^(lse_in-m) + e^(l_blk-m)).
+ * The block output is the normalised fp32 accumulator of the kernel (one
+ * rounding less than va3d_ring_merge, which reads a bf16 o_blk).
+ * (Anthology record sota-390: ring context parallelism for long videos;
+ * log-sum-exp merging of softmax blocks over disjoint key sets.)
+ *   q_rot       device bf16 [B, heads, n_rows, head_dim], read only.
+ *   k, v        device bf16 [B, heads, n_keys, head_dim], read only.
+ *   acc         device fp32 [B, heads, n_rows, head_dim], read (unless first)
+ *               and written.
+ *   lse_in      device fp32 [B, heads, n_rows] (natural log); NULL when first;
+ *               must not alias lse_out.
+ *   lse_out     device fp32 [B, heads, n_rows], written.
+ *   out         device bf16 [B, heads, n_rows, head_dim] receiving the merged
+ *               output as well (the last block), or NULL.
+ *   softmax_scale  <= 0 selects 1/sqrt(head_dim).
+ * Asynchronous on `stream`.  Every query tile runs whole (no workspace).
+ * Errors: VA3D_ERR_INVALID, _UNSUPPORTED, _ALIGNMENT, _DEVICE, _CUDA.
+ */
+int va3d_ring_attend(const va3d_bf16 *q_rot, const va3d_bf16 *k, const va3d_bf16 *v, float *acc,
+                     const float *lse_in, float *lse_out, va3d_bf16 *out, int B, int heads,
+                     int n_rows, int n_keys, int head_dim, float softmax_scale, int first,
+                     void *stream);
 
 #ifdef __cplusplus
 }

@@ -240,13 +240,17 @@ class FakeRingBackend(FakeBackend):
     def ring_merge(self, o_blk, lse_blk, acc, lse_in, lse_out, first, out=None):
         self.calls.append(("merge", first, out is not None))
 
+    def ring_attend(self, q_rot, k, v, acc, lse_in, lse_out, first, out=None):
+        self.calls.append(("attend", first, out is not None))
+
 
 def test_ring_call_sequence():
     """Rank 1 of 3: neighbours mapped (next = rank 2, previous = rank 0); per
     call one load, then per step the free wait and pass (not at the last
-    step), the product, the free signal to the previous rank, the merge (the
-    last one writes the output) and the full wait (not at the last step),
-    with counts that grow across calls."""
+    step), the product with its merge into the accumulator (one call; the
+    last one writes the output), the free signal to the previous rank and
+    the full wait (not at the last step), with counts that grow across
+    calls."""
     import torch
     from full_spatiotemporal_attention_b200.ring import RingAttention
     import full_spatiotemporal_attention_b200 as va
@@ -264,7 +268,7 @@ def test_ring_call_sequence():
         for s in range(3):
             if s < 2:
                 expect += [("wait", own, 1, (c - 1) * 3 + s), ("pass", own, nxt, s % 2)]
-            expect += [("product",), ("free_signal", prv), ("merge", s == 0, s == 2)]
+            expect += [("attend", s == 0, s == 2), ("free_signal", prv)]
             if s < 2:
                 expect += [("wait", own, 0, (c - 1) * 2 + s + 1)]
         assert fake.calls == expect

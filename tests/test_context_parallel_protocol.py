@@ -209,9 +209,8 @@ def ring_calls(world_size, rank, calls):
     import full_spatiotemporal_attention_b200 as va
 
     class Recorder(FakeRingBackend):
-        def attn_cross_fwd(self, q, k, v, out=None, lse=None, workspace=None):
-            self.calls.append(("product", 0 if k is self.owner.kbuf[0] else 1))
-            return out, lse
+        def ring_attend(self, q_rot, k, v, acc, lse_in, lse_out, first, out=None):
+            self.calls.append(("attend", 0 if k is self.owner.kbuf[0] else 1))
 
     fake = Recorder(rank)
     handles = [f"handle-of-{0x10000 * (j + 1):#x}".encode() for j in range(world_size)]
@@ -255,21 +254,19 @@ def ring_program(P, rank, calls):
                 write_end(w, (nxt, "kv", 1 - buf), state["passing"])
                 w.add(nxt, "full")
             prog += [begin, end]
-        elif c[0] == "product":
+        elif c[0] == "attend":
+            # the block product reads the buffer; its merge ends the step
             buf = c[1]
             def begin(w, buf=buf):
                 assert buf == state["step"] % 2
                 read_begin(w, (rank, "kv", buf), (state["call"], (rank - state["step"]) % P))
             def end(w, buf=buf):
                 read_end(w, (rank, "kv", buf))
+                state["step"] += 1
             prog += [begin, end]
         elif c[0] == "free_signal":
             assert region_rank(c[1]) == (rank - 1) % P
             prog.append(lambda w: w.add((rank - 1) % P, "free"))
-        elif c[0] == "merge":
-            def merged(w):
-                state["step"] += 1
-            prog.append(merged)
         else:
             raise AssertionError(f"unexpected call {c}")
     return prog

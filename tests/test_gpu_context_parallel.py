@@ -249,9 +249,12 @@ def test_wait_gives_up_and_reports(va):
 
 # ------------------------------------------------------------ ring form
 
-def emulate_ring(va, w, world, calls=1):
+def emulate_ring(va, w, world, calls=1, fold=True):
     """`calls` ring calls of `world` emulated ranks, every rank's launches in
     turn on one stream (each wait launched after the signals it counts).
+    fold: each step is one va3d_ring_attend (merge in the attention kernel's
+    epilogue, as RingAttention runs it); otherwise attn_cross_fwd with its
+    LSE, then va3d_ring_merge.
     Returns the assembled output [B, heads, N, 128] and LSE [B, heads, N]."""
     q, k, v = (dev(x) for x in si.qkv(w))
     g = vgrid(va, w)
@@ -283,12 +286,18 @@ def emulate_ring(va, w, world, calls=1):
                         va.ring_wait(regions[r], va.RING_FREE, (c - 1) * world + s, world, B, H, N)
                         va.ring_pass(regions[r], regions[(r + 1) % world], cur, world, B, H, N)
                 for r in range(world):
-                    va.attn_cross_fwd(q_rot[r], kbuf[r][cur], vbuf[r][cur], out=o_blk[r],
-                                      lse=lse_blk[r], workspace=ws)
+                    if fold:
+                        va.ring_attend(q_rot[r], kbuf[r][cur], vbuf[r][cur], acc[r],
+                                       lse[(s + 1) % 2][r], lse[s % 2][r], first=(s == 0),
+                                       out=out[r] if s == world - 1 else None)
+                    else:
+                        va.attn_cross_fwd(q_rot[r], kbuf[r][cur], vbuf[r][cur], out=o_blk[r],
+                                          lse=lse_blk[r], workspace=ws)
+                        va.ring_merge(o_blk[r], lse_blk[r], acc[r], lse[(s + 1) % 2][r],
+                                      lse[s % 2][r], first=(s == 0),
+                                      out=out[r] if s == world - 1 else None)
                     if world > 1:
                         va.ring_free(regions[(r - 1) % world])
-                    va.ring_merge(o_blk[r], lse_blk[r], acc[r], lse[(s + 1) % 2][r], lse[s % 2][r],
-                                  first=(s == 0), out=out[r] if s == world - 1 else None)
                 if s < world - 1:
                     for r in range(world):
                         va.ring_wait(regions[r], va.RING_FULL, (c - 1) * (world - 1) + s + 1, world,
@@ -313,6 +322,18 @@ RING_CASES = [(si.WORKLOADS["tiny"], 2), (si.WORKLOADS["c17f480"], 4),
 @pytest.mark.parametrize("w,world", RING_CASES, ids=lambda x: getattr(x, "name", str(x)))
 def test_ring_matches_oracle(va, w, world):
     o, lse = emulate_ring(va, w, world)
+    qb, kb, vb = si.qkv(w)
+    ref, ref_lse = oracle.attention(qb, kb, vb, ogrid(w), want_lse=True)
+    check(host(o).reshape(ref.shape), ref, f"ring {w.name} x{world}")
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(ref_lse.shape), ref_lse, atol=2e-3, rtol=0)
+
+
+@pytest.mark.parametrize("w,world", [RING_CASES[1], RING_CASES[3], RING_CASES[4]],
+                         ids=lambda x: getattr(x, "name", str(x)))
+def test_ring_two_call_merge_matches_oracle(va, w, world):
+    """The separate merge kernel (attn_cross_fwd + va3d_ring_merge) computes
+    the same as the folded step."""
+    o, lse = emulate_ring(va, w, world, fold=False)
     qb, kb, vb = si.qkv(w)
     ref, ref_lse = oracle.attention(qb, kb, vb, ogrid(w), want_lse=True)
     check(host(o).reshape(ref.shape), ref, f"ring {w.name} x{world}")

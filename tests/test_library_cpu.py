@@ -256,6 +256,14 @@ def test_ring_region_layout_and_bad_arguments(va):
     assert lib.va3d_ring_merge(p, p, p, None, q16, None, 1, 2, 16, 0, None) == -1      # no lse_in
     assert lib.va3d_ring_merge(ctypes.c_void_p(p.value + 2), p, p, p, ctypes.c_void_p(p.value + 64),
                                None, 1, 2, 16, 0, None) == -3
+    # folded step: the same LSE rules, sizes and alignment, checked before any launch
+    assert lib.va3d_ring_attend(p, p, p, p, p, p, None, 1, 2, 16, 16, 128, 0.0, 0, None) == -1
+    assert lib.va3d_ring_attend(p, p, p, p, None, q16, None, 1, 2, 16, 16, 128, 0.0, 0, None) == -1
+    assert lib.va3d_ring_attend(p, p, p, p, None, None, None, 1, 2, 16, 16, 128, 0.0, 1, None) == -1
+    assert lib.va3d_ring_attend(p, p, p, p, None, q16, None, 1, 2, 16, 16, 64, 0.0, 1, None) == -2
+    assert lib.va3d_ring_attend(p, p, p, p, None, q16, None, 1, 2, 0, 16, 128, 0.0, 1, None) == -1
+    assert lib.va3d_ring_attend(ctypes.c_void_p(p.value + 2), p, p, p, None, q16, None, 1, 2, 16, 16,
+                                128, 0.0, 1, None) == -3
 
 
 def test_binding_has_no_cpu_path(va):
