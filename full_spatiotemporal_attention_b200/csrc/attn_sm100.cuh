@@ -125,8 +125,7 @@ struct AttnArgs {
     float2 *part_ml;   // [split tiles][2][256] (row maximum in log2 units, row sum)
     int *part_count;   // [split tiles] halves finished
     float scale_log2;  // softmax scale * log2(e)
-    int rope_q;        // 1: rotate Q tiles with the table
-    const float2 *rope_tab;
+    int rope_q;        // 1: rotate Q tiles by 3D RoPE (hardware sine and cosine)
     __nv_bfloat16 *o;
     float *lse;        // may be null
     RopeParams rp;

@@ -87,12 +87,15 @@ __global__ void rope_table_kernel(float2 *__restrict__ tab, int *__restrict__ ze
 // y = RoPE(x) for [BH, N, 128] bf16.  One thread per (token, 16-byte chunk)
 // computes the four angles of its chunk once and applies them to the chunk
 // in every (batch, head) row, four rows in flight at a time.  x may equal y.
+// It also clears `n_zero` ints at `zero` (the split-tail counters of the
+// attention launch that follows on the same stream).
 constexpr int kRopeThreads = 256;
 
 __global__ void __launch_bounds__(kRopeThreads)
 rope_apply_kernel(const uint4 *x, uint4 *y, long long N, int BH,
-                  const __grid_constant__ RopeParams rp) {
+                  const __grid_constant__ RopeParams rp, int *zero, int n_zero) {
     const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gid < n_zero) zero[gid] = 0;
     if (gid >= N * 16) return;
     const int n = static_cast<int>(gid >> 4);
     const int c = static_cast<int>(gid & 15);

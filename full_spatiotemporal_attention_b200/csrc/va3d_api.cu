@@ -198,7 +198,39 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // [BH, N, 128] bf16 viewed as a 3D tensor (dim, row, bh); boxes of
 // 64 columns x box_rows rows with the 128-byte swizzle; rows past N read as zero.
+// Encoding is a pure host computation of (base, N, BH, box_rows), so the
+// last maps encoded are kept (a small direct-mapped cache under a mutex).
+int encode_map(CUtensorMap *map, const void *base, int N, int BH, int box_rows);
+
+struct MapSlot {
+    const void *base;
+    int N, BH, box_rows;
+    CUtensorMap map;
+};
+constexpr int kMapSlots = 64;
+MapSlot g_map_slots[kMapSlots] = {};
+std::mutex g_map_mutex;
+
 int make_map(CUtensorMap *map, const void *base, int N, int BH, int box_rows) {
+    const uintptr_t key = reinterpret_cast<uintptr_t>(base) ^ (static_cast<uintptr_t>(N) * 0x9E3779B1u) ^
+                          (static_cast<uintptr_t>(BH) << 7) ^ static_cast<uintptr_t>(box_rows);
+    MapSlot &slot = g_map_slots[(key ^ (key >> 17) ^ (key >> 31)) % kMapSlots];
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    if (slot.base == base && slot.N == N && slot.BH == BH && slot.box_rows == box_rows && base != nullptr) {
+        *map = slot.map;
+        return VA3D_OK;
+    }
+    const int rc = encode_map(map, base, N, BH, box_rows);
+    if (rc != VA3D_OK) return rc;
+    slot.base = base;
+    slot.N = N;
+    slot.BH = BH;
+    slot.box_rows = box_rows;
+    slot.map = *map;
+    return VA3D_OK;
+}
+
+int encode_map(CUtensorMap *map, const void *base, int N, int BH, int box_rows) {
     auto fn = encode_fn();
     if (fn == nullptr) return VA3D_ERR_CUDA;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(N),
@@ -255,11 +287,14 @@ int launch_table(float2 *tab, int *zero, int n_zero, const RopeParams &rp, cudaS
     return launch_status();
 }
 
-int launch_rope(const void *x, void *y, int BH, int N, const RopeParams &rp, cudaStream_t st) {
+// zero, n_zero: split-tail counters of the attention launch that follows,
+// cleared by the same launch (optional).
+int launch_rope(const void *x, void *y, int BH, int N, const RopeParams &rp, cudaStream_t st,
+                int *zero = nullptr, int n_zero = 0) {
     const long long threads = static_cast<long long>(N) * 16;
     const long long blocks = (threads + kRopeThreads - 1) / kRopeThreads;
     rope_apply_kernel<<<static_cast<unsigned>(blocks), kRopeThreads, 0, st>>>(
-        static_cast<const uint4 *>(x), static_cast<uint4 *>(y), N, BH, rp);
+        static_cast<const uint4 *>(x), static_cast<uint4 *>(y), N, BH, rp, zero, n_zero);
     return launch_status();
 }
 
@@ -319,7 +354,6 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
     a.q_blocks = (seg_len + nq * fa::BM - 1) / (nq * fa::BM);
     a.scale_log2 = static_cast<float>(scale * kLog2e);
     a.rope_q = rope_q ? 1 : 0;
-    a.rope_tab = tab;
     a.o = static_cast<__nv_bfloat16 *>(o);
     a.lse = lse;
     a.rp = rp;
@@ -444,9 +478,13 @@ size_t required_workspace_bytes(int B, int heads, int N, const va3d_grid_t *grid
 // split_optional: accept a workspace that holds only the required part (the
 // built-in scratch of the no-allocation entry point); the public entry
 // points ask for the full va3d_workspace_bytes().
+// need_table: build the angle table (only the temporal pass reads it; the
+// attention kernel forms its angles with the hardware sine and cosine).
+// The split-tail counters are cleared by whichever of the table kernel or the
+// key pre-pass runs, else by a clearing launch of the table kernel alone.
 int prepare(const void *q, const void *k, const void *v, int B, int heads, int N, int head_dim,
             const va3d_grid_t *grid, float softmax_scale, unsigned flags, void *workspace,
-            size_t workspace_bytes, bool need_k_rot, cudaStream_t st, Prepared *out,
+            size_t workspace_bytes, bool need_k_rot, bool need_table, cudaStream_t st, Prepared *out,
             bool split_optional = false) {
     int rc;
     if ((rc = check_sizes(B, heads, N, head_dim)) != VA3D_OK) return rc;
@@ -467,16 +505,23 @@ int prepare(const void *q, const void *k, const void *v, int B, int heads, int N
     size_t used = required_workspace_bytes(B, heads, N, grid, flags);
     out->split = split_scratch(used < workspace_bytes ? static_cast<uint8_t *>(workspace) + used : nullptr,
                                used < workspace_bytes ? workspace_bytes - used : 0);
-    if ((rc = launch_table(static_cast<float2 *>(workspace), out->split.count, out->split.capacity,
-                           out->rp, st)) != VA3D_OK)
-        return rc;
+    const bool prepass = !(flags & VA3D_K_ROTATED) && need_k_rot;
+    if (need_table || (!prepass && out->split.capacity > 0)) {
+        RopeParams tab_rp = out->rp;
+        if (!need_table) tab_rp.tab_entries = 0;   // counters only
+        if ((rc = launch_table(static_cast<float2 *>(workspace), prepass ? nullptr : out->split.count,
+                               prepass ? 0 : out->split.capacity, tab_rp, st)) != VA3D_OK)
+            return rc;
+    }
     if (flags & VA3D_K_ROTATED) {
         out->k_rot = k;
     } else if (!need_k_rot) {
         out->k_rot = nullptr;
     } else {
         void *kr = static_cast<uint8_t *>(workspace) + table_bytes(grid);
-        if ((rc = launch_rope(k, kr, B * heads, N, out->rp, st)) != VA3D_OK) return rc;
+        if ((rc = launch_rope(k, kr, B * heads, N, out->rp, st, out->split.count, out->split.capacity)) !=
+            VA3D_OK)
+            return rc;
         out->k_rot = kr;
     }
     return VA3D_OK;
@@ -556,7 +601,7 @@ int full_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, va3d_bf
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Prepared p;
     int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
-                     workspace_bytes, true, st, &p, split_optional);
+                     workspace_bytes, true, false, st, &p, split_optional);
     if (rc != VA3D_OK) return rc;
     return launch_attn(q, p.k_rot, v, o, lse, B * heads, N, N, N, N, 1, true, p.rp, p.tab, p.scale,
                        p.split, st);
@@ -589,7 +634,7 @@ int attn_factorized_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Prepared p;
     int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
-                     workspace_bytes, o_spatial != nullptr, st, &p);
+                     workspace_bytes, o_spatial != nullptr, o_temporal != nullptr, st, &p);
     if (rc != VA3D_OK) return rc;
     if (o_spatial != nullptr) {
         rc = launch_attn(q, p.k_rot, v, o_spatial, nullptr, B * heads, N, N, p.rp.HW, p.rp.HW,
@@ -648,7 +693,7 @@ int attn_window_fwd(const va3d_bf16 *q, const va3d_bf16 *k, const va3d_bf16 *v, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Prepared p;
     int rc = prepare(q, k, v, B, heads, N, head_dim, grid, softmax_scale, flags, workspace,
-                     workspace_bytes, true, st, &p);
+                     workspace_bytes, true, false, st, &p);
     if (rc != VA3D_OK) return rc;
     const int win[3] = {win_t, win_h, win_w};
     const int vol = win_t * win_h * win_w;
