@@ -18,6 +18,7 @@
 #include "rope.cuh"
 #include "attn_sm100.cuh"
 #include "attn_temporal.cuh"
+#include "attn_temporal_tc.cuh"
 #include "selftest.cuh"
 #include "ulysses.cuh"
 #include "ring.cuh"
@@ -66,7 +67,11 @@ int check_sizes(int B, int heads, int N, int head_dim) {
 // dynamic shared-memory limit already granted to each kernel), looked up
 // once per device under a mutex instead of on every call.
 constexpr int kMaxDevices = 64;
-enum KernelSlot { K_ATTN2, K_ATTN1, K_TEMP32R, K_TEMP32K, K_TEMP64R, K_TEMP64K, NUM_KERNEL_SLOTS };
+enum KernelSlot {
+    K_ATTN2, K_ATTN1, K_TEMP64R, K_TEMP64K,
+    K_TTC0,   // temporal_tc_kernel<R, raw>: K_TTC0 + 2 * log2(R / 8) + (raw ? 0 : 1)
+    NUM_KERNEL_SLOTS = K_TTC0 + 6
+};
 
 struct DeviceInfo {
     int state;                     // 0 unknown, 1 sm_100, 2 other architecture
@@ -202,32 +207,67 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // last maps encoded are kept (a small direct-mapped cache under a mutex).
 int encode_map(CUtensorMap *map, const void *base, int N, int BH, int box_rows);
 
+// The temporal pass's view of [BH, T*HW, 128] bf16: a 4D tensor (dim, frame,
+// position, bh) whose frames are HW rows apart; boxes of 64 dims x R frames x
+// P positions (frames past T and positions past HW read as zero), 128-byte
+// swizzle.
+int encode_map_tp(CUtensorMap *map, const void *base, int T, int HW, int BH, int R, int P);
+
 struct MapSlot {
     const void *base;
     int N, BH, box_rows;
+    int T, HW, P;   // temporal-pass maps (box_rows = R); 0 for the 3D maps
     CUtensorMap map;
 };
 constexpr int kMapSlots = 64;
 MapSlot g_map_slots[kMapSlots] = {};
 std::mutex g_map_mutex;
 
-int make_map(CUtensorMap *map, const void *base, int N, int BH, int box_rows) {
+// Cached encoding: (T, HW, P) = (0, 0, 0) selects the 3D map of
+// encode_map, otherwise the temporal-pass map of encode_map_tp (N = T * HW).
+int make_map_any(CUtensorMap *map, const void *base, int N, int BH, int box_rows, int T, int HW, int P) {
     const uintptr_t key = reinterpret_cast<uintptr_t>(base) ^ (static_cast<uintptr_t>(N) * 0x9E3779B1u) ^
-                          (static_cast<uintptr_t>(BH) << 7) ^ static_cast<uintptr_t>(box_rows);
+                          (static_cast<uintptr_t>(BH) << 7) ^ static_cast<uintptr_t>(box_rows) ^
+                          (static_cast<uintptr_t>(P) << 13);
     MapSlot &slot = g_map_slots[(key ^ (key >> 17) ^ (key >> 31)) % kMapSlots];
     std::lock_guard<std::mutex> lock(g_map_mutex);
-    if (slot.base == base && slot.N == N && slot.BH == BH && slot.box_rows == box_rows && base != nullptr) {
+    if (slot.base == base && slot.N == N && slot.BH == BH && slot.box_rows == box_rows && slot.T == T &&
+        slot.HW == HW && slot.P == P && base != nullptr) {
         *map = slot.map;
         return VA3D_OK;
     }
-    const int rc = encode_map(map, base, N, BH, box_rows);
+    const int rc = P == 0 ? encode_map(map, base, N, BH, box_rows)
+                          : encode_map_tp(map, base, T, HW, BH, box_rows, P);
     if (rc != VA3D_OK) return rc;
     slot.base = base;
     slot.N = N;
     slot.BH = BH;
     slot.box_rows = box_rows;
+    slot.T = T;
+    slot.HW = HW;
+    slot.P = P;
     slot.map = *map;
     return VA3D_OK;
+}
+
+int make_map(CUtensorMap *map, const void *base, int N, int BH, int box_rows) {
+    return make_map_any(map, base, N, BH, box_rows, 0, 0, 0);
+}
+
+int encode_map_tp(CUtensorMap *map, const void *base, int T, int HW, int BH, int R, int P) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return VA3D_ERR_CUDA;
+    const cuuint64_t row = static_cast<cuuint64_t>(kHeadDim) * 2;   // bytes per token row
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(T),
+                          static_cast<cuuint64_t>(HW), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[3] = {row * static_cast<cuuint64_t>(HW), row,
+                             row * static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(HW)};
+    cuuint32_t box[4] = {64, static_cast<cuuint32_t>(R), static_cast<cuuint32_t>(P), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VA3D_OK : VA3D_ERR_CUDA;
 }
 
 int encode_map(CUtensorMap *map, const void *base, int N, int BH, int box_rows) {
@@ -425,7 +465,8 @@ int launch_temporal_t(const tp::TemporalArgs &a, cudaStream_t st) {
     const int warps = std::max(1, std::min(tp::Cfg<MAXT>::kMaxWarps, budget / warp_bytes));
     const int smem = table_bytes + warps * warp_bytes;
     const int per_sm = std::max(1, std::min(4, (216 * 1024) / smem));
-    constexpr int slot = MAXT <= 32 ? (kRawK ? K_TEMP32R : K_TEMP32K) : (kRawK ? K_TEMP64R : K_TEMP64K);
+    static_assert(MAXT == 64, "T' <= 32 runs on the tensor-core pass");
+    constexpr int slot = kRawK ? K_TEMP64R : K_TEMP64K;
     if ((rc = grant_smem(reinterpret_cast<const void *>(tp::temporal_kernel<MAXT, kRawK>), slot, smem)) !=
         VA3D_OK)
         return rc;
@@ -434,6 +475,39 @@ int launch_temporal_t(const tp::TemporalArgs &a, cudaStream_t st) {
     const long long blocks = std::min<long long>(need, static_cast<long long>(sms) * per_sm);
     tp::temporal_kernel<MAXT, kRawK><<<static_cast<unsigned>(blocks), warps * 32, smem, st>>>(a);
     return launch_status();
+}
+
+// Tensor-core temporal pass (T' <= 32): one persistent block per SM, each
+// block's two groups taking alternate tiles of P positions.
+template <int R, bool kRawK>
+int launch_temporal_tc_t(const tp::TemporalArgs &a, cudaStream_t st) {
+    constexpr int P = tpc::Geo<R>::P;
+    int sms = 0, rc;
+    if ((rc = device_sms(&sms)) != VA3D_OK) return rc;
+    CUtensorMap mq, mk, mv, mo;
+    if ((rc = make_map_any(&mq, a.q, a.N, a.BH, R, a.T, a.HW, P)) != VA3D_OK) return rc;
+    if ((rc = make_map_any(&mk, a.k, a.N, a.BH, R, a.T, a.HW, P)) != VA3D_OK) return rc;
+    if ((rc = make_map_any(&mv, a.v, a.N, a.BH, R, a.T, a.HW, P)) != VA3D_OK) return rc;
+    if ((rc = make_map_any(&mo, a.o, a.N, a.BH, R, a.T, a.HW, P)) != VA3D_OK) return rc;
+    const int smem = tpc::smem_bytes(a.T, a.rp.pe_t);
+    constexpr int slot = K_TTC0 + 2 * (R == 8 ? 0 : (R == 16 ? 1 : 2)) + (kRawK ? 0 : 1);
+    if ((rc = grant_smem(reinterpret_cast<const void *>(tpc::temporal_tc_kernel<R, kRawK>), slot, smem)) !=
+        VA3D_OK)
+        return rc;
+    const long long tiles = static_cast<long long>(a.BH) * ((a.HW + P - 1) / P);
+    if (tiles >= (1ll << 30)) return VA3D_ERR_UNSUPPORTED;   // tile indices are 32-bit
+    const long long blocks = std::min<long long>(tiles, sms);
+    tpc::temporal_tc_kernel<R, kRawK><<<static_cast<unsigned>(blocks), tpc::kThreads, smem, st>>>(mq, mk, mv, mo, a);
+    return launch_status();
+}
+
+template <bool kRawK>
+int launch_temporal_tc(const tp::TemporalArgs &a, cudaStream_t st) {
+    switch (tpc::rows_per_position(a.T)) {
+    case 8: return launch_temporal_tc_t<8, kRawK>(a, st);
+    case 16: return launch_temporal_tc_t<16, kRawK>(a, st);
+    default: return launch_temporal_tc_t<32, kRawK>(a, st);
+    }
 }
 
 // k is the raw key tensor (rotated here) unless k_rotated.
@@ -453,8 +527,7 @@ int launch_temporal(const void *q, const void *k, bool k_rotated, const void *v,
     a.rope_k = k_rotated ? 0 : 1;
     a.rope_tab = tab;
     a.rp = rp;
-    if (rp.T <= 32)
-        return k_rotated ? launch_temporal_t<32, false>(a, st) : launch_temporal_t<32, true>(a, st);
+    if (rp.T <= 32) return k_rotated ? launch_temporal_tc<false>(a, st) : launch_temporal_tc<true>(a, st);
     return k_rotated ? launch_temporal_t<64, false>(a, st) : launch_temporal_t<64, true>(a, st);
 }
 

@@ -72,7 +72,11 @@ SMALL = [si.WORKLOADS["tiny"], si.WORKLOADS["c17f480"],
 
 FACTORISED_SMALL = [si.WORKLOADS["tiny"], si.WORKLOADS["c17f480"], custom("f_odd", 3, 5, 17, heads=3),
                     custom("f_t1", 1, 9, 15), custom("f_t33", 33, 2, 3), custom("f_t64", 64, 1, 5),
-                    custom("f_hw1", 7, 1, 1), custom("f_b2", 4, 6, 7, batch=2)]
+                    custom("f_hw1", 7, 1, 1), custom("f_b2", 4, 6, 7, batch=2),
+                    # frames padded to 16, 24 and 32 rows per position (8, 5 and 4
+                    # positions per 128-row tile), position counts not a multiple
+                    custom("f_t12", 12, 3, 5), custom("f_t21", 21, 2, 7, dims=(16, 56, 56)),
+                    custom("f_t29", 29, 3, 3, heads=3)]
 
 LARGE = ["c81f480", "c81f720", "joint720", "refimg720"]
 
@@ -170,6 +174,25 @@ def test_repeat_calls_are_deterministic(va):
 def test_factorised_all_rows(va, w):
     q, k, v = si.qkv(w)
     os_, ot = va.attn_factorized_fwd(dev(q), dev(k), dev(v), vgrid(va, w))
+    shape = (w.batch * w.heads, w.N, 128)
+    check(host(os_).reshape(shape), oracle.attention(q, k, v, ogrid(w), mode="spatial"),
+          f"spatial {w.name}")
+    check(host(ot).reshape(shape), oracle.attention(q, k, v, ogrid(w), mode="temporal"),
+          f"temporal {w.name}")
+    assert va.device_error() == 0
+
+
+@pytest.mark.parametrize("w", [si.WORKLOADS["c17f480"], custom("r_t12", 12, 3, 5),
+                               custom("r_t21", 21, 2, 7), custom("r_t29", 29, 3, 3, heads=3),
+                               custom("r_t40", 40, 2, 3)], ids=lambda w: w.name)
+def test_factorised_with_prerotated_keys(va, w):
+    """Keys turned by rope3d_apply and passed with k_rotated: the temporal
+    pass then turns Q in full and runs all of QK^T in scaled fp16."""
+    q, k, v = si.qkv(w)
+    g = vgrid(va, w)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    kr = va.rope3d_apply(kd, g)
+    os_, ot = va.attn_factorized_fwd(qd, kr, vd, g, k_rotated=True)
     shape = (w.batch * w.heads, w.N, 128)
     check(host(os_).reshape(shape), oracle.attention(q, k, v, ogrid(w), mode="spatial"),
           f"spatial {w.name}")
