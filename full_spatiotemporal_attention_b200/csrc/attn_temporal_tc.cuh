@@ -32,7 +32,8 @@
 // even and odd tiles) through its own Q/K stage, V stage and TMEM columns, so
 // one group's loads and products overlap the other's arithmetic.  Thread 0 of
 // a group issues its products and refills its stages: Q/K as soon as S is
-// done, V as soon as O is done.  Every mbarrier wait is bounded; a group
+// done, V once the previous tile's O store has read the stage (O is staged
+// in the V stage and written by TMA store).  Every mbarrier wait is bounded; a group
 // leaves its loop together (the barrier that closes each step ANDs the
 // threads' wait results) and drains what it issued before TMEM is freed.
 #pragma once
