@@ -23,10 +23,10 @@
 // range needs turning.  Each thread turns the first ceil16(d_t) dims of its
 // row of Q and K in place as fp16; the QK^T k-steps over those dims run as
 // fp16 x fp16 products, the rest as bf16 x bf16 on the untouched inputs (exact
-// products), all into one fp32 accumulator.  If the tile's turned values leave
-// fp16's comfortable range, the tile is redone with all dims in fp16 under
-// per-tile powers of two; keys that come rotated always take that form (Q
-// turned in full).
+// products), all into one fp32 accumulator.  Keys that come rotated: Q is
+// turned in full and K converted, both fp16, and all of QK^T runs in fp16.
+// If the values written leave fp16's comfortable range, the tile is redone
+// with all dims in fp16 under per-tile powers of two.
 //
 // Roles: two groups of four warps, each running its own tiles (the CTA's
 // even and odd tiles) through its own Q/K stage, V stage and TMEM columns, so
@@ -308,8 +308,33 @@ temporal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 v_ph = ph;
             }
         }
-        // ---- raw keys: turn the t range of this row of Q and K in place (fp16)
+        // ---- raw keys: turn the t range of this row of Q and K in place (fp16).
+        // Keys that come rotated: turn all of this row of Q and convert K,
+        // both unscaled fp16.  mx tracks the largest value written.
         float mx = 0.f;
+        if (!kRawK && good && valid) {
+            const int hh = pos / a.rp.W, ww = pos - hh * a.rp.W;
+#pragma unroll 2
+            for (int c = 0; c < 16; ++c) {
+                const uint32_t off = chunk_off(r, c);
+                const uint4 xq = *reinterpret_cast<const uint4 *>(sq + off);
+                const uint4 xk = *reinterpret_cast<const uint4 *>(sk + off);
+                float2 cq[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int p = 4 * c + e;
+                    // h and w angles: the same address across a position's rows
+                    cq[e] = p < a.rp.pe_t ? tab[f * TS + p]
+                                          : __ldg(&a.rope_tab[table_index(a.rp, p, 0, hh, ww)]);
+                }
+                *reinterpret_cast<uint4 *>(sq + off) =
+                    make_uint4(tp::rot_f16_max(xq.x, cq[0], mx), tp::rot_f16_max(xq.y, cq[1], mx),
+                               tp::rot_f16_max(xq.z, cq[2], mx), tp::rot_f16_max(xq.w, cq[3], mx));
+                *reinterpret_cast<uint4 *>(sk + off) =
+                    make_uint4(tp::cvt_f16_max(xk.x, mx), tp::cvt_f16_max(xk.y, mx),
+                               tp::cvt_f16_max(xk.z, mx), tp::cvt_f16_max(xk.w, mx));
+            }
+        }
         if (kRawK && good && valid) {
             const float2 *ang = tab + f * TS;
             for (int c = 0; c < nc; c += 2) {
@@ -346,27 +371,27 @@ temporal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
         fence_proxy_async_smem();
         if (!named_and(bid, 128, good)) break;
-        int f16_steps = nc / 2;   // k-steps of QK^T over fp16 operands
+        int f16_steps = kRawK ? nc / 2 : 8;   // k-steps of QK^T over fp16 operands
         int eq = 0, ek = 0;
-        bool full = !kRawK;
-        if constexpr (kRawK) {
-            const float m = fmaxf(fmaxf(red[g * 8], red[g * 8 + 2]), fmaxf(red[g * 8 + 4], red[g * 8 + 6]));
-            full = !tp::fp16_range_ok(m);
-        }
+        const bool full = !tp::fp16_range_ok(
+            fmaxf(fmaxf(red[g * 8], red[g * 8 + 2]), fmaxf(red[g * 8 + 4], red[g * 8 + 6])));
         if (full) {
-            // all dims in fp16 under per-tile powers of two, from the inputs
-            // in global memory (the t chunks in shared memory may be turned);
-            // the early bf16 products finish reading the stage first
+            // the values written left fp16's comfortable range: all dims in
+            // fp16 under per-tile powers of two, from the rows in global memory
+            // (the stage holds turned values), once the early bf16 products
+            // have read the stage
             if constexpr (kRawK)
                 good = __all_sync(0xffffffffu, mbar_wait(bar(B_E0 + g), ph, abort_flag,
                                                          VA3D_DEVERR_TIMEOUT_SOFTMAX)) && good;
             const __nv_bfloat16 *gq = a.q + rowofs, *gk = a.k + rowofs;
+            auto row_q = [&](int c) -> uint4 { return tp::ldg_stream(gq + 8 * c); };
+            auto row_k = [&](int c) -> uint4 { return tp::ldg_stream(gk + 8 * c); };
             float mq = 0.f, mk = 0.f;
             if (valid) {
 #pragma unroll 4
                 for (int c = 0; c < 16; ++c) {
-                    mq = absmax8(tp::ldg_stream(gq + 8 * c), mq);
-                    mk = absmax8(tp::ldg_stream(gk + 8 * c), mk);
+                    mq = absmax8(row_q(c), mq);
+                    mk = absmax8(row_k(c), mk);
                 }
             }
             const uint32_t wq = __reduce_max_sync(0xffffffffu, __float_as_uint(mq));
@@ -390,10 +415,11 @@ temporal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const float sq_scale = tp::pow2f(eq), sk_scale = tp::pow2f(ek);
             if (valid) {
                 const int hh = pos / a.rp.W, ww = pos - hh * a.rp.W;
+#pragma unroll 2
                 for (int c = 0; c < 16; ++c) {
-                    const uint4 xq = tp::ldg_stream(gq + 8 * c);
-                    const uint4 xk = tp::ldg_stream(gk + 8 * c);
-                    float2 cq[4], ck[4];
+                    const uint4 xq = row_q(c);
+                    const uint4 xk = row_k(c);
+                    float2 cq[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int p = 4 * c + e;
@@ -402,20 +428,31 @@ temporal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                             an = tab[f * TS + p];
                         else if (kRawK)
                             an = make_float2(1.f, 0.f);
-                        else
-                            an = a.rope_tab[table_index(a.rp, p, 0, hh, ww)];
+                        else   // same address across a position's rows: a broadcast
+                            an = __ldg(&a.rope_tab[table_index(a.rp, p, 0, hh, ww)]);
                         cq[e] = make_float2(an.x * sq_scale, an.y * sq_scale);
-                        // keys: turned by t only when raw, else converted as they are
-                        const float2 bk = kRawK && p < a.rp.pe_t ? an : make_float2(1.f, 0.f);
-                        ck[e] = make_float2(bk.x * sk_scale, bk.y * sk_scale);
                     }
                     const uint32_t off = chunk_off(r, c);
                     *reinterpret_cast<uint4 *>(sq + off) =
                         make_uint4(tp::rot_f16(xq.x, cq[0]), tp::rot_f16(xq.y, cq[1]),
                                    tp::rot_f16(xq.z, cq[2]), tp::rot_f16(xq.w, cq[3]));
-                    *reinterpret_cast<uint4 *>(sk + off) =
-                        make_uint4(tp::rot_f16(xk.x, ck[0]), tp::rot_f16(xk.y, ck[1]),
-                                   tp::rot_f16(xk.z, ck[2]), tp::rot_f16(xk.w, ck[3]));
+                    if constexpr (kRawK) {
+                        // raw keys: t pairs turned, the others converted
+                        float2 ck[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int p = 4 * c + e;
+                            const float2 bk = p < a.rp.pe_t ? tab[f * TS + p] : make_float2(1.f, 0.f);
+                            ck[e] = make_float2(bk.x * sk_scale, bk.y * sk_scale);
+                        }
+                        *reinterpret_cast<uint4 *>(sk + off) =
+                            make_uint4(tp::rot_f16(xk.x, ck[0]), tp::rot_f16(xk.y, ck[1]),
+                                       tp::rot_f16(xk.z, ck[2]), tp::rot_f16(xk.w, ck[3]));
+                    } else {
+                        *reinterpret_cast<uint4 *>(sk + off) =
+                            make_uint4(tp::cvt_f16(xk.x, sk_scale), tp::cvt_f16(xk.y, sk_scale),
+                                       tp::cvt_f16(xk.z, sk_scale), tp::cvt_f16(xk.w, sk_scale));
+                    }
                 }
             }
             fence_proxy_async_smem();
