@@ -131,9 +131,11 @@ struct AttnArgs {
     RopeParams rp;
     // Local 3D windows (win != 0): segment s is window s of the grid in
     // (t, h, w) raster order of windows, its rows the window's tokens in
-    // (dt, dh, dw) raster order.  Rows are gathered token by token from the
-    // natural-order tensors below (no TMA), and O and LSE rows are written
-    // back to the tokens' natural positions.
+    // (dt, dh, dw) raster order; O and LSE rows are written back to the
+    // tokens' natural positions.  win == 2 (window width a multiple of 8 that
+    // divides 128): a tile's rows arrive as runs of win_w consecutive tokens,
+    // one TMA box each.  win == 1: rows are gathered token by token from the
+    // natural-order tensors below.
     int win;
     int win_t, win_h, win_w;   // window size
     int nwin_h, nwin_w;        // windows along h and w
@@ -256,7 +258,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(bar(B_QREADY1), BM);
         // full barriers: one TMA arrival with its byte count, or one arrival
         // per gathering thread in window mode
-        const uint32_t full_count = a.win ? 64u : 1u;
+        const uint32_t full_count = a.win == 1 ? 64u : 1u;
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(B_KFULL0 + s), full_count);
             mbar_init(bar(B_KEMPTY0 + s), 1);
@@ -292,7 +294,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // (16-byte cp.async into the same swizzled layout TMA produces), two
         // tiles in flight; after its copies land a thread fences them for the
         // tensor core's proxy and arrives on the tile's full barrier.
-        if (a.win) {
+        if (a.win == 1) {
             const int lt = threadIdx.x - kGather * 32;   // 0..63
             auto gather = [&](const __nv_bfloat16 *src, uint32_t dst, int j) {
 #pragma unroll
@@ -363,7 +365,74 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
     } else if (warp == kLoad) {
         // ------------------------------------------------------------ loader
-        if (lane == 0 && !a.win) {
+        if (a.win == 2) {
+            // -------------------------------------------- window runs loader
+            // A tile's rows arrive as runs of win_w consecutive tokens, one box
+            // of the win_w-row maps each; lane u issues run u of every tile.
+            // Runs past the window repeat its last run (those rows are masked
+            // as keys and not stored as queries).
+            const int runs = BM / a.win_w;
+            const int n_runs = a.seg_len / a.win_w;
+            const int origin = window_token(a, seg, 0);
+            auto load_runs = [&](const CUtensorMap *map, uint32_t dst, uint32_t fbar, int local0) {
+                if (lane < runs) {
+                    const int run = min(local0 / a.win_w + lane, n_runs - 1);
+                    const int dt = run / a.win_h, dh = run - dt * a.win_h;
+                    const int row = origin + dt * a.rp.HW + dh * a.rp.W;
+                    for (int hf = 0; hf < 2; ++hf)
+                        tma_load_3d(dst + hf * kHalfBytes + lane * a.win_w * 128, map, fbar, hf * 64, row, bh);
+                }
+            };
+            if (lane == 0) {
+                tma_prefetch_desc(&tmQ);
+                tma_prefetch_desc(&tmK);
+                tma_prefetch_desc(&tmV);
+                mbar_arrive_expect_tx(bar(B_QFULL), NQ * kTileBytes);
+            }
+            __syncwarp();
+            for (int i = 0; i < NQ; ++i)
+                load_runs(&tmQ, sbase + OFF_Q + i * kTileBytes, bar(B_QFULL), q0 - seg_start + i * BM);
+            int k_issued = 0, v_issued = 0;
+            bool ok = true;
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = stg(j);
+                const uint32_t ph = phs(j);
+                if (j >= kStages &&
+                    !(ok = __all_sync(0xffffffffu, mbar_wait(bar(B_KEMPTY0 + s), ph ^ 1, abort_flag,
+                                                             VA3D_DEVERR_TIMEOUT_LOAD))))
+                    break;
+                if (lane == 0) mbar_arrive_expect_tx(bar(B_KFULL0 + s), kTileBytes);
+                __syncwarp();
+                load_runs(&tmK, sbase + OFF_K + s * kTileBytes, bar(B_KFULL0 + s), (j0 + j) * BN);
+                k_issued = j + 1;
+                if (j >= kStages &&
+                    !(ok = __all_sync(0xffffffffu, mbar_wait(bar(B_VEMPTY0 + s), ph ^ 1, abort_flag,
+                                                             VA3D_DEVERR_TIMEOUT_LOAD))))
+                    break;
+                if (lane == 0) mbar_arrive_expect_tx(bar(B_VFULL0 + s), kTileBytes);
+                __syncwarp();
+                load_runs(&tmV, sbase + OFF_V + s * kTileBytes, bar(B_VFULL0 + s), (j0 + j) * BN);
+                v_issued = j + 1;
+            }
+            const int k_first = k_issued > kStages ? k_issued - kStages : 0;
+            const int v_first = v_issued > kStages ? v_issued - kStages : 0;
+            if (ok) {
+                for (int j = k_first; j < k_issued && ok; ++j)
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar(B_KEMPTY0 + stg(j)), phs(j), abort_flag,
+                                                           VA3D_DEVERR_TIMEOUT_LOAD));
+                for (int j = v_first; j < v_issued && ok; ++j)
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar(B_VEMPTY0 + stg(j)), phs(j), abort_flag,
+                                                           VA3D_DEVERR_TIMEOUT_LOAD));
+            }
+            if (!ok) {
+                // Let the copies already in flight land before the CTA exits.
+                mbar_wait_drain(bar(B_QFULL), 0);
+                for (int j = k_first; j < k_issued; ++j)
+                    mbar_wait_drain(bar(B_KFULL0 + stg(j)), phs(j));
+                for (int j = v_first; j < v_issued; ++j)
+                    mbar_wait_drain(bar(B_VFULL0 + stg(j)), phs(j));
+            }
+        } else if (lane == 0 && !a.win) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
@@ -521,7 +590,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // natural token index of this row (differs from n only for windows)
         const int n_out = a.win && n < seg_end ? window_token(a, seg, n - seg_start) : n;
         bool ok = true;
-        if (a.win) {
+        if (a.win == 1) {
             // gather this row of Q itself (256 contiguous bytes) into the
             // swizzled tile; rows past the window are zero
             uint8_t *tile = smem + OFF_Q + g * kTileBytes;
@@ -547,7 +616,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QFULL), 0, abort_flag,
                                                    VA3D_DEVERR_TIMEOUT_SOFTMAX));
             if (ok) {
-                if (a.rope_q) rope_q_row(smem + OFF_Q + g * kTileBytes, r, n, a);
+                if (a.rope_q) rope_q_row(smem + OFF_Q + g * kTileBytes, r, n_out, a);
                 fence_proxy_async_smem();
                 mbar_arrive(bar(g ? B_QREADY1 : B_QREADY0));
             }

@@ -379,9 +379,13 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
                 const int *win = nullptr, const RingMerge *merge = nullptr) {
     CUtensorMap mq, mk, mv;
     int rc;
-    if ((rc = make_map(&mq, q, N, BH, fa::BM)) != VA3D_OK) return rc;
-    if ((rc = make_map(&mk, k_rot, Nkv, BH, fa::BN)) != VA3D_OK) return rc;
-    if ((rc = make_map(&mv, v, Nkv, BH, fa::BN)) != VA3D_OK) return rc;
+    // windows whose width is a multiple of 8 dividing 128 load their rows as
+    // TMA boxes of one run (win_w consecutive tokens) each
+    const bool win_runs = win != nullptr && win[2] % 8 == 0 && fa::BM % win[2] == 0;
+    const int qrows = win_runs ? win[2] : fa::BM, krows = win_runs ? win[2] : fa::BN;
+    if ((rc = make_map(&mq, q, N, BH, qrows)) != VA3D_OK) return rc;
+    if ((rc = make_map(&mk, k_rot, Nkv, BH, krows)) != VA3D_OK) return rc;
+    if ((rc = make_map(&mv, v, Nkv, BH, krows)) != VA3D_OK) return rc;
     fa::AttnArgs a;
     std::memset(&a, 0, sizeof a);
     a.N = N;
@@ -398,7 +402,7 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
     a.lse = lse;
     a.rp = rp;
     if (win != nullptr) {
-        a.win = 1;
+        a.win = win_runs ? 2 : 1;
         a.win_t = win[0];
         a.win_h = win[1];
         a.win_w = win[2];
