@@ -149,6 +149,10 @@ struct AttnArgs {
     float *acc;
     const float *lse_in;
     float *lse_out;
+    // O written by TMA store from the group's Q tile: 1 = one box of 128
+    // rows per half (map: [n_seg * BH] segments of seg_len rows), 2 = one box
+    // per window run (map: [BH, N] rows, boxes of win_w rows); 0 = row stores
+    int o_tma;
 };
 
 // Natural token index of row `local` of window `seg`.
@@ -215,7 +219,8 @@ __device__ __forceinline__ void rope_q_row(uint8_t *tile, int r, int n, const At
 template <int NQ>
 __global__ void __launch_bounds__(KCfg<NQ>::kThreads, KCfg<NQ>::kMinBlocks)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                const __grid_constant__ AttnArgs a) {
     using C = KCfg<NQ>;
     constexpr int kStages = C::kStages;
     constexpr int OFF_Q = C::OFF_Q, OFF_K = C::OFF_K, OFF_V = C::OFF_V;
@@ -783,6 +788,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 if (valid) a.lse_out[row] = lo2 * 0.69314718055994531f;
             } else if (!split) {
+                // O rows staged in this group's Q tile (its products are all
+                // done) for the TMA store below, or written row by row
+                uint8_t *stage = smem + OFF_Q + g * kTileBytes;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t ov[32];
@@ -794,11 +802,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     for (int e = 0; e < 16; ++e)
                         pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l,
                                             __uint_as_float(ov[2 * e + 1]) * inv_l);
-                    if (valid) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
-                                                        pk[4 * e + 3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const uint4 w4 = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        const int cc = c * 4 + e;   // 16-byte chunk of the row
+                        if (a.o_tma)
+                            *reinterpret_cast<uint4 *>(stage + (cc >> 3) * kHalfBytes + r * 128 +
+                                                       (((cc & 7) ^ (r & 7)) << 4)) = w4;
+                        else if (valid)
+                            dst[cc] = w4;
                     }
                 }
                 if (a.lse != nullptr && valid)
@@ -859,6 +871,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     if (a.lse != nullptr && valid)
                         a.lse[static_cast<size_t>(bh) * a.N + n_out] =
                             (m_max + log2f(w_s + w_o)) * 0.69314718055994531f;
+                }
+            }
+        }
+        if (a.o_tma && !split && !a.merge) {
+            // every row of the group is staged (or a wait gave up: then no
+            // store); the store clips rows past the segment (o_tma == 1: one
+            // box of 128 rows per half) or stores only the window's runs
+            // (o_tma == 2: one box of win_w rows per run, natural positions)
+            fence_proxy_async_smem();
+            const bool all_ok = named_and(1 + g, BM, ok);
+            const uint32_t stage = sbase + OFF_Q + g * kTileBytes;
+            if (all_ok && (warp & 3) == 0) {
+                if (a.o_tma == 1) {
+                    if (lane == 0) {
+                        for (int hf = 0; hf < 2; ++hf)
+                            tma_store_3d(&tmO, stage + hf * kHalfBytes, hf * 64,
+                                         q0 - seg_start + g * BM, bh * a.n_seg + seg);
+                        bulk_commit_group();
+                        bulk_wait_group0();
+                    }
+                } else {
+                    const int runs = BM / a.win_w;
+                    const int run = (q0 - seg_start + g * BM) / a.win_w + lane;
+                    if (lane < runs && run < a.seg_len / a.win_w) {
+                        const int dt = run / a.win_h, dh = run - dt * a.win_h;
+                        const int row = window_token(a, seg, 0) + dt * a.rp.HW + dh * a.rp.W;
+                        for (int hf = 0; hf < 2; ++hf)
+                            tma_store_3d(&tmO, stage + hf * kHalfBytes + lane * a.win_w * 128, hf * 64,
+                                         row, bh);
+                        bulk_commit_group();
+                        bulk_wait_group0();
+                    }
                 }
             }
         }

@@ -419,6 +419,19 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
         a.lse_in = merge->lse_in;
         a.lse_out = merge->lse_out;
     }
+    // O by TMA store: segments that tile the rows (boxes clipped at each
+    // segment's end), or window runs; the ring merge writes rows itself
+    CUtensorMap mo;
+    std::memset(&mo, 0, sizeof mo);
+    if (merge == nullptr && o != nullptr) {
+        if (win_runs) {
+            if ((rc = make_map(&mo, o, N, BH, win[2])) != VA3D_OK) return rc;
+            a.o_tma = 2;
+        } else if (win == nullptr && static_cast<long long>(seg_len) * n_seg == N) {
+            if ((rc = make_map(&mo, o, seg_len, n_seg * BH, fa::BM)) != VA3D_OK) return rc;
+            a.o_tma = 1;
+        }
+    }
     // One CTA per SM.  If the last wave of tiles would fill at most half of the
     // SMs and every tile has at least two 128-key steps, each of its tiles is
     // covered by two units over half of the keys instead.
@@ -444,14 +457,14 @@ int launch_attn(const void *q, const void *k_rot, const void *v, void *o, float 
                              C::kSmemBytes)) != VA3D_OK)
             return rc;
         fa::attn_fwd_kernel<2><<<static_cast<unsigned>(units), C::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, a);
+            mq, mk, mv, mo, a);
     } else {
         using C = fa::KCfg<1>;
         if ((rc = grant_smem(reinterpret_cast<const void *>(fa::attn_fwd_kernel<1>), K_ATTN1,
                              C::kSmemBytes)) != VA3D_OK)
             return rc;
         fa::attn_fwd_kernel<1><<<static_cast<unsigned>(units), C::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, a);
+            mq, mk, mv, mo, a);
     }
     return launch_status();
 }
