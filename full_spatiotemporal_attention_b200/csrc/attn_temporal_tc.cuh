@@ -69,7 +69,13 @@ __host__ __device__ inline int tab_stride(int pe_t) { return tab_pairs(pe_t) + 2
 
 __host__ __device__ inline int tab_bytes(int T, int pe_t) { return T * tab_stride(pe_t) * 8; }
 
-__host__ inline int smem_bytes(int T, int pe_t) { return 1024 + OFF_TAB + tab_bytes(T, pe_t) + kMiscBytes; }
+// Keys that come rotated: per warp, the h and w angles of its (up to four)
+// positions, 64 pairs each.
+constexpr int kHwBytes = 8 * 4 * 64 * 8;
+
+__host__ inline int smem_bytes(int T, int pe_t, bool raw_k) {
+    return 1024 + OFF_TAB + tab_bytes(T, pe_t) + kMiscBytes + (raw_k ? 0 : kHwBytes);
+}
 
 __host__ __device__ constexpr int rows_per_position(int T) { return T <= 8 ? 8 : (T <= 16 ? 16 : 32); }
 
@@ -184,6 +190,7 @@ temporal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int off_misc = OFF_TAB + tab_bytes(T, a.rp.pe_t);
     float2 *tab = reinterpret_cast<float2 *>(smem + OFF_TAB);
     uint8_t *misc = smem + off_misc;
+    float2 *hw_ang = reinterpret_cast<float2 *>(misc + kMiscBytes);   // [warp][position][pair]
     auto bar = [&](int i) -> uint32_t { return sbase + off_misc + 8 * i; };
     float *red = reinterpret_cast<float *>(misc + 128);   // [group][warp][2]
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 200);
@@ -312,28 +319,52 @@ temporal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         // Keys that come rotated: turn all of this row of Q and convert K,
         // both unscaled fp16.  mx tracks the largest value written.
         float mx = 0.f;
-        if (!kRawK && good && valid) {
+        if (!kRawK && good) {
+            // the h and w angles of this row's position, computed once by its
+            // R rows (hardware sine and cosine: absolute error ~1e-5 at the
+            // largest angles of the pages' grids, far below fp16's rounding of
+            // the turned values)
             const int hh = pos / a.rp.W, ww = pos - hh * a.rp.W;
-#pragma unroll 2
-            for (int c = 0; c < 16; ++c) {
-                const uint32_t off = chunk_off(r, c);
-                const uint4 xq = *reinterpret_cast<const uint4 *>(sq + off);
-                const uint4 xk = *reinterpret_cast<const uint4 *>(sk + off);
-                float2 cq[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int p = 4 * c + e;
-                    // h and w angles: the same address across a position's rows
-                    cq[e] = p < a.rp.pe_t ? tab[f * TS + p]
-                                          : __ldg(&a.rope_tab[table_index(a.rp, p, 0, hh, ww)]);
-                }
-                *reinterpret_cast<uint4 *>(sq + off) =
-                    make_uint4(tp::rot_f16_max(xq.x, cq[0], mx), tp::rot_f16_max(xq.y, cq[1], mx),
-                               tp::rot_f16_max(xq.z, cq[2], mx), tp::rot_f16_max(xq.w, cq[3], mx));
-                *reinterpret_cast<uint4 *>(sk + off) =
-                    make_uint4(tp::cvt_f16_max(xk.x, mx), tp::cvt_f16_max(xk.y, mx),
-                               tp::cvt_f16_max(xk.z, mx), tp::cvt_f16_max(xk.w, mx));
+            const float fh = static_cast<float>(hh), fw = static_cast<float>(ww);
+            float2 *ha = hw_ang + (warp * 4 + kofs) * 64;
+            for (int p = a.rp.pe_t + f; p < 64; p += R) {
+                float2 cs;
+                __sincosf((p < a.rp.pe_h ? fh : fw) * a.rp.inv_freq[p], &cs.y, &cs.x);
+                ha[p] = cs;
             }
+            __syncwarp();
+        }
+        if (!kRawK && good && valid) {
+            const float2 *ha = hw_ang + (warp * 4 + kofs) * 64;
+            const float2 *tt = tab + f * TS;
+            float m2[2] = {0.f, 0.f};
+            for (int c = 0; c < 16; c += 2) {
+                // two chunks per pass: all loads first
+                uint4 xq[2], xk[2];
+                float2 cq[2][4];
+                uint32_t off[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    off[u] = chunk_off(r, c + u);
+                    xq[u] = *reinterpret_cast<const uint4 *>(sq + off[u]);
+                    xk[u] = *reinterpret_cast<const uint4 *>(sk + off[u]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int p = 4 * (c + u) + e;
+                        cq[u][e] = p < a.rp.pe_t ? tt[p] : ha[p];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    *reinterpret_cast<uint4 *>(sq + off[u]) = make_uint4(
+                        tp::rot_f16_max(xq[u].x, cq[u][0], m2[u]), tp::rot_f16_max(xq[u].y, cq[u][1], m2[u]),
+                        tp::rot_f16_max(xq[u].z, cq[u][2], m2[u]), tp::rot_f16_max(xq[u].w, cq[u][3], m2[u]));
+                    *reinterpret_cast<uint4 *>(sk + off[u]) = make_uint4(
+                        tp::cvt_f16_max(xk[u].x, m2[u]), tp::cvt_f16_max(xk[u].y, m2[u]),
+                        tp::cvt_f16_max(xk[u].z, m2[u]), tp::cvt_f16_max(xk[u].w, m2[u]));
+                }
+            }
+            mx = fmaxf(m2[0], m2[1]);
         }
         if (kRawK && good && valid) {
             const float2 *ang = tab + f * TS;

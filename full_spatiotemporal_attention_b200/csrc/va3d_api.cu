@@ -506,7 +506,7 @@ int launch_temporal_tc_t(const tp::TemporalArgs &a, cudaStream_t st) {
     if ((rc = make_map_any(&mk, a.k, a.N, a.BH, R, a.T, a.HW, P)) != VA3D_OK) return rc;
     if ((rc = make_map_any(&mv, a.v, a.N, a.BH, R, a.T, a.HW, P)) != VA3D_OK) return rc;
     if ((rc = make_map_any(&mo, a.o, a.N, a.BH, R, a.T, a.HW, P)) != VA3D_OK) return rc;
-    const int smem = tpc::smem_bytes(a.T, a.rp.pe_t);
+    const int smem = tpc::smem_bytes(a.T, a.rp.pe_t, kRawK);
     constexpr int slot = K_TTC0 + 2 * (R == 8 ? 0 : (R == 16 ? 1 : 2)) + (kRawK ? 0 : 1);
     if ((rc = grant_smem(reinterpret_cast<const void *>(tpc::temporal_tc_kernel<R, kRawK>), slot, smem)) !=
         VA3D_OK)
