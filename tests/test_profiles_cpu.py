@@ -25,7 +25,7 @@ def _fields(path):
 
 def test_profiles_exist_for_the_main_kernels():
     names = {os.path.basename(p) for p in _summaries()}
-    for kernel in ("attn_fwd_kernel", "rope_apply_kernel", "temporal_kernel"):
+    for kernel in ("attn_fwd_kernel", "rope_apply_kernel", "temporal_tc_kernel"):
         assert any(n.startswith(kernel) for n in names), kernel
     assert os.path.exists(os.path.join(ROOT, "profiles", "launches_c81f480.md"))
 
