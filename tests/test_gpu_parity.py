@@ -236,6 +236,26 @@ def test_temporal_pass_at_extreme_magnitudes(va, k):
     assert va.device_error() == 0
 
 
+@pytest.mark.parametrize("k", [-14, 14])
+@pytest.mark.parametrize("w", [si.WORKLOADS["c17f480"], custom("x_t21", 21, 4, 7)], ids=lambda w: w.name)
+@pytest.mark.parametrize("rotated", [False, True], ids=["raw_keys", "rotated_keys"])
+def test_temporal_pass_fallback_for_both_key_forms(va, k, w, rotated):
+    """Queries times 2^k and keys times 2^-k push the values written as fp16
+    out of range, so every tile takes the scaled fallback: with raw keys and
+    with keys that come rotated (rope3d_apply of the scaled keys), on 8- and
+    32-row position tiles."""
+    q, kk, v = si.qkv(w)
+    q, kk = _scale_bits(q, k), _scale_bits(kk, -k)
+    g = vgrid(va, w)
+    kd = dev(kk)
+    if rotated:
+        kd = va.rope3d_apply(kd, g)
+    _, ot = va.attn_factorized_fwd(dev(q), kd, dev(v), g, spatial=False, k_rotated=rotated)
+    ref = oracle.attention(q, kk, v, ogrid(w), mode="temporal")
+    check(host(ot).reshape(ref.shape), ref, f"temporal {w.name} 2^{k} rotated={rotated}")
+    assert va.device_error() == 0
+
+
 def test_factorised_single_pass_outputs(va):
     w = si.WORKLOADS["tiny"]
     q, k, v = (dev(x) for x in si.qkv(w))
