@@ -878,7 +878,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             // every row of the group is staged (or a wait gave up: then no
             // store); the store clips rows past the segment (o_tma == 1: one
             // box of 128 rows per half) or stores only the window's runs
-            // (o_tma == 2: one box of win_w rows per run, natural positions)
+            // (o_tma == 2: one box of win_w rows per run, natural positions).
+            // The CTA may leave once the store has read shared memory; its
+            // writes complete before the grid does.
             fence_proxy_async_smem();
             const bool all_ok = named_and(1 + g, BM, ok);
             const uint32_t stage = sbase + OFF_Q + g * kTileBytes;
@@ -889,7 +891,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                             tma_store_3d(&tmO, stage + hf * kHalfBytes, hf * 64,
                                          q0 - seg_start + g * BM, bh * a.n_seg + seg);
                         bulk_commit_group();
-                        bulk_wait_group0();
+                        bulk_wait_group_read0();
                     }
                 } else {
                     const int runs = BM / a.win_w;
@@ -901,7 +903,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                             tma_store_3d(&tmO, stage + hf * kHalfBytes + lane * a.win_w * 128, hf * 64,
                                          row, bh);
                         bulk_commit_group();
-                        bulk_wait_group0();
+                        bulk_wait_group_read0();
                     }
                 }
             }

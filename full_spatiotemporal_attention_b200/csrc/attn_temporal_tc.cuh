@@ -596,7 +596,7 @@ temporal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // products and loads this group issued finish before TMEM and shared
     // memory are given up
     if (leader) {
-        bulk_wait_group0();
+        bulk_wait_group_read0();   // the last O store has read its stage
         mma_commit(bar(B_DRAIN0 + g));
         mbar_wait_drain(bar(B_DRAIN0 + g), 0);
         if (qk_out) mbar_wait_drain(bar(B_QK0 + g), qk_ph);
