@@ -256,6 +256,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int j0 = split && part ? n_kv_all / 2 : 0;
     const int j1 = split && !part ? n_kv_all / 2 : n_kv_all;
     const int n_kv = j1 - j0;   // key tiles of this unit; local step jj = j - j0
+    // Two query tiles, unless the second lies wholly past the segment (the
+    // last block of a segment shorter than it): then only tile 0 is computed
+    // and the second softmax group idles.  Split units keep both (their merge
+    // counts the rows of both tiles).
+    const bool two = NQ == 2 && (split || q0 + BM < seg_end);
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_QFULL), 1);
@@ -516,13 +521,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             };
 
             bool ok = mbar_wait(bar(B_QREADY0), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA) &&
-                      (NQ == 1 || mbar_wait(bar(B_QREADY1), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA)) &&
+                      (!two || mbar_wait(bar(B_QREADY1), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA)) &&
                       mbar_wait(bar(B_KFULL0), 0, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
             if (ok) {
                 tc_fence_after();
                 issue_s(0, 0);
                 mma_commit(bar(B_SFULL0));
-                if constexpr (NQ == 2) {
+                if (two) {
                     issue_s(1, 0);
                     mma_commit(bar(B_SFULL1));
                 }
@@ -546,7 +551,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 // one query tile: V's stage is free after this product.  (Its
                 // release must not wait for the next QK^T: with one stage the
                 // gathering loader publishes that K tile only after refilling V.)
-                if constexpr (NQ == 1) mma_commit(bar(B_VEMPTY0 + s));
+                if (!two) mma_commit(bar(B_VEMPTY0 + s));
                 if (more) {
                     ok = mbar_wait(bar(B_KFULL0 + s2), ph2, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
                     if (!ok) break;
@@ -554,7 +559,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     issue_s(0, s2);
                     mma_commit(bar(B_SFULL0));
                 }
-                if constexpr (NQ == 2) {
+                if (two) {
                     ok = mbar_wait(bar(B_PHALF1), j & 1, abort_flag, VA3D_DEVERR_TIMEOUT_MMA);
                     if (!ok) break;
                     tc_fence_after();
@@ -566,7 +571,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     mma_commit(bar(B_VEMPTY0 + s));
                 }
                 if (more) {
-                    if constexpr (NQ == 2) {
+                    if (two) {
                         issue_s(1, s2);
                         mma_commit(bar(B_SFULL1));
                     }
@@ -582,7 +587,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
         }
     }
-    } else {
+    } else if (warp < 4 || two) {
         regs_raise<C::kSoftmaxRegs>();
         // ---------------------------------------------------------- softmax
         const int g = warp >> 2;                  // query tile of this group
