@@ -459,6 +459,14 @@ def bench_ours(args, rank, world, local):
                          "frac": round(2 * tensor_bytes / (rope_ms / 1e3) / 1e9 / peak_gbs, 4)},
         "clocks": clocks,
     }
+    # The kernel is bound by the SM clock (tensor and softmax pipes), which
+    # the power cap sets: its time in clock cycles is the clock-free figure.
+    if clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
+        line["roofline"]["clock_normalised"] = {
+            "kernel_mcycles": round(attn_ms * clocks["sm_mhz"] / 1e3, 4),
+            "achieved_at_max_clock": round(achieved * clocks["sm_max_mhz"] / clocks["sm_mhz"], 2),
+            "note": "kernel time x median SM clock of the timed region; achieved scaled to sm_max_mhz",
+        }
 
     if world == 1 and not args.no_extras:
         line["extras"] = extras(va, device, stream, peak_tf, peak_gbs)
