@@ -44,7 +44,10 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="c81f480")
-    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--e2e-steps", type=int, default=None,
+                   help="steps of the end-to-end loop (default: --steps); the pipelined loop's "
+                        "first upload and last download are not overlapped, so they are spread "
+                        "over these steps")
     p.add_argument("--no-extras", action="store_true", help="skip the secondary measurements")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per head for cpu_baseline")
@@ -56,7 +59,10 @@ def parse_args():
     p.add_argument("--case", choices=["temporal720", "spatial720", "window720", "cross720"],
                    help="run only this secondary kernel (warm-up + --steps launches, one "
                         "JSON line); a small, single-kernel command for profilers")
-    return p.parse_args()
+    args = p.parse_args()
+    if args.e2e_steps is None:
+        args.e2e_steps = args.steps
+    return args
 
 
 def peaks():
