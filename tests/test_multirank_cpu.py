@@ -92,3 +92,13 @@ def test_reference_arm_runs_on_rank_zero_only(tmp_path):
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_e2e_loop_runs_as_many_steps_as_the_timed_loop(monkeypatch):
+    # the pipelined end-to-end loop spreads its one unoverlapped upload and
+    # download over its steps, so by default it runs --steps of them
+    import bench
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "7"])
+    assert bench.parse_args().e2e_steps == 7
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "7", "--e2e-steps", "3"])
+    assert bench.parse_args().e2e_steps == 3
