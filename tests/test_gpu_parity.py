@@ -1,7 +1,7 @@
 """Parity of the sm_100a kernels (through the C ABI) with the fp64 oracle.
 
-Bar (per BASELINE's stated tolerance for bf16 outputs with fp32
-accumulation): max-abs error <= 1.5e-2 and mean-abs error <= 2e-3; in
+Bar (the tolerance set for bf16 outputs with fp32 accumulation):
+max-abs error <= 1.5e-2 and mean-abs error <= 2e-3; in
 addition the relative L2 error must stay <= 2e-2, which is the meaningful
 gate at large N where outputs are small.  Small workloads compare every
 row; the full-size workloads (the configuration the bench times) compare
